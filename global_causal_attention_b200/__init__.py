@@ -1,0 +1,177 @@
+"""Python binding of the ZGCM-1 attention-core library (libgswa.so, sm_100a).
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels behind the C ABI declared in include/gswa.h.  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing or no sm_100 device is current, the calls raise.
+
+Entry points (same names as the C ABI):
+  gswa_fwd       gated sliding-window attention forward  (ZGCM-1 §2.1, Figure 3)
+  full_attn_fwd  full causal attention of the global layers (§2.1)
+  gswa_bwd, full_attn_bwd, gswa_decode, full_decode  (see include/gswa.h)
+  gswa_kv_cache_bytes  KV-cache footprint closed form (§2.3)
+  gswa_check_status    read and clear the device status word
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgswa.so")
+
+OK = 0
+ERRORS = {
+    -1: "INVALID_ARG", -2: "UNSUPPORTED_SHAPE", -3: "MISALIGNED", -4: "WORKSPACE_TOO_SMALL",
+    -5: "LAUNCH", -6: "TIMEOUT", -7: "UNIMPLEMENTED", -8: "NO_DEVICE",
+}
+OP_GSWA_FWD, OP_FULL_FWD, OP_GSWA_BWD, OP_FULL_BWD, OP_GSWA_DECODE, OP_FULL_DECODE = range(6)
+
+
+class GswaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({strerror(code)})")
+
+
+class Shape(ctypes.Structure):
+    """Mirror of gswa_shape_t."""
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("rope_dims", ctypes.c_int32), ("cache_len", ctypes.c_int32),
+                ("rope_base", ctypes.c_double), ("eps", ctypes.c_float),
+                ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run global_causal_attention_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, I, U = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.c_int, ctypes.c_size_t
+        sig = {
+            "gswa_fwd": [S, P, P, P, P, P, P, P, P, P, U, P],
+            "full_attn_fwd": [S, P, P, P, P, P, P, P, P, U, P],
+            "gswa_bwd": [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, U, P],
+            "full_attn_bwd": [S, P, P, P, P, P, P, P, P, P, P, P, P, P, U, P],
+            "gswa_decode": [S, P, P, P, P, P, P, P, P, P, P, P, U, P],
+            "full_decode": [S, P, P, P, P, P, P, P, P, P, U, P],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = I
+        L.gswa_workspace_bytes.argtypes = [I, S]
+        L.gswa_workspace_bytes.restype = U
+        L.gswa_kv_cache_bytes.argtypes = [I, I, I, I, I, I, ctypes.c_int64]
+        L.gswa_kv_cache_bytes.restype = ctypes.c_int64
+        L.gswa_check_status.argtypes = [P]
+        L.gswa_check_status.restype = I
+        L.gswa_strerror.argtypes = [I]
+        L.gswa_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().gswa_strerror(code).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise GswaError(rc, what)
+
+
+def make_shape(B, T, Hq, Hkv, D=128, window=128, rope_dims=42, rope_base=1e4, eps=1e-6,
+               scale=None, cache_len=0) -> Shape:
+    return Shape(B, T, Hq, Hkv, D, window, rope_dims, cache_len, rope_base, eps,
+                 1.0 / math.sqrt(D) if scale is None else scale)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(*ts):
+    torch = _torch()
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on the GPU")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    return torch
+
+
+def gswa_fwd(q, k, v, g, wq, wk, *, window=128, rope_dims=42, rope_base=1e4, eps=1e-6,
+             scale=None, y=None, lse=None, stream=None):
+    """Gated SWA forward.  q, g [B,T,Hq,D], k, v [B,T,Hkv,D], wq, wk [D] (bf16, cuda).
+    Returns (y [B,T,Hq,D] bf16, lse [B,Hq,T] f32)."""
+    torch = _dev(q, k, v, g, wq, wk, y, lse)
+    B, T, Hq, D = q.shape
+    s = make_shape(B, T, Hq, k.shape[2], D, window, rope_dims, rope_base, eps, scale)
+    if y is None:
+        y = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    _check(lib().gswa_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
+                          _ptr(wk), _ptr(y), _ptr(lse), None, 0, _stream(stream)), "gswa_fwd")
+    return y, lse
+
+
+def full_attn_fwd(q, k, v, wq, wk, *, rope_dims=42, rope_base=1e4, eps=1e-6, scale=None,
+                  y=None, lse=None, workspace=None, stream=None):
+    """Full causal forward of a global layer (no gate).  Returns (y, lse)."""
+    torch = _dev(q, k, v, wq, wk, y, lse)
+    B, T, Hq, D = q.shape
+    s = make_shape(B, T, Hq, k.shape[2], D, 0, rope_dims, rope_base, eps, scale)
+    if y is None:
+        y = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    ws, nb = _workspace(OP_FULL_FWD, s, workspace, q.device)
+    _check(lib().full_attn_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk),
+                               _ptr(y), _ptr(lse), _ptr(ws), nb, _stream(stream)),
+           "full_attn_fwd")
+    return y, lse
+
+
+def _workspace(op, s, workspace, device):
+    torch = _torch()
+    need = lib().gswa_workspace_bytes(op, ctypes.byref(s))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace, (workspace.numel() * workspace.element_size() if workspace is not None else 0)
+
+
+def workspace_bytes(op, shape: Shape) -> int:
+    return int(lib().gswa_workspace_bytes(op, ctypes.byref(shape)))
+
+
+def gswa_kv_cache_bytes(n_global_layers, n_window_layers, window, Hkv, D, bytes_per_elem, T) -> int:
+    return int(lib().gswa_kv_cache_bytes(n_global_layers, n_window_layers, window, Hkv, D,
+                                         bytes_per_elem, T))
+
+
+def gswa_check_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib().gswa_check_status(_stream(stream)))

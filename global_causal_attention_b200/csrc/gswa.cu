@@ -1,0 +1,261 @@
+// gswa.cu -- C ABI of the ZGCM-1 attention core (declared in include/gswa.h).
+//
+// Host-side argument validation, TMA tensor-map encoding and kernel launch.
+// One translation unit: every kernel of the library is included here so that
+// they share the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gswa.h"
+#include "ptx.cuh"
+#include "swa_fwd.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int status = GSWA_OK;
+    int num_sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device set-up (compute capability check, kernel attributes, SM count),
+// done once per device under a lock.
+int device_setup(int *num_sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GSWA_ERR_NO_DEVICE;
+    if (dev < 0 || dev >= kMaxDevices) return GSWA_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        d.ready = true;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            d.status = GSWA_ERR_NO_DEVICE;
+        } else if (major != 10 || minor != 0) {
+            d.status = GSWA_ERR_NO_DEVICE;  // built for sm_100a only
+        } else if (cudaFuncSetAttribute(gswa::swa::swa_fwd_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)gswa::swa::kSmemBytes) != cudaSuccess) {
+            d.status = GSWA_ERR_LAUNCH;
+        }
+        if (d.status == GSWA_OK && g_encode == nullptr) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                d.status = GSWA_ERR_LAUNCH;
+            else
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    *num_sms = d.num_sms;
+    return d.status;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D bf16 tensor map over [B, T, H, D] (innermost first: D, H, T, B) with a
+// {64, box_h, box_t, 1} box and the 128-byte swizzle the MMA descriptors use.
+int encode_bthd(CUtensorMap *m, const void *base, int B, int T, int H, int D, int box_h, int box_t)
+{
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_t, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
+}
+
+// Shape checks common to every entry point.
+int check_common(const gswa_shape_t *s)
+{
+    if (s == nullptr) return GSWA_ERR_INVALID_ARG;
+    if (s->B < 0 || s->T < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->D <= 0) return GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale))
+        return GSWA_ERR_INVALID_ARG;
+    if (s->D != 128) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->Hq != 4 * s->Hkv) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1)) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    return GSWA_OK;
+}
+
+void fill_theta(double *theta, int R, double base)
+{
+    for (int p = 0; p < 64; ++p)
+        theta[p] = (p < R / 2) ? std::pow(base, -2.0 * (double)p / (double)R) : 0.0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
+             const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
+             size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    int rc = check_common(s);
+    if (rc != GSWA_OK) return rc;
+    if (s->window < 1 || s->window > 128) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)s->B * s->T == 0) return GSWA_OK;
+    if (!q || !k || !v || !g || !w_q || !w_k || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(y) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+
+    CUtensorMap tq, tk, tv, tg, ty;
+    if (encode_bthd(&tq, q, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&tg, g, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&ty, y, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&tk, k, s->B, s->T, s->Hkv, s->D, 1, 32) ||
+        encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, 32))
+        return GSWA_ERR_INVALID_ARG;
+
+    gswa::swa::Params p;
+    std::memset(&p, 0, sizeof p);
+    p.B = s->B;
+    p.T = s->T;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.window = s->window;
+    p.R = s->rope_dims;
+    p.nsteps = (s->T + gswa::swa::kTok - 1) / gswa::swa::kTok;
+    p.units = (long long)s->B * s->Hkv * p.nsteps;
+    p.eps = s->eps;
+    p.sl2 = s->scale * 1.4426950408889634f;
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.lse = lse;
+    fill_theta(p.theta, s->rope_dims, s->rope_base);
+
+    const long long grid = p.units < num_sms ? p.units : num_sms;
+    gswa::swa::swa_fwd_kernel<<<(unsigned)grid, gswa::swa::kThreads, gswa::swa::kSmemBytes,
+                                static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tg, ty, p);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
+int full_attn_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
+                  const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
+                  size_t workspace_bytes, void *stream)
+{
+    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)y; (void)lse;
+    (void)workspace; (void)workspace_bytes; (void)stream;
+    return GSWA_ERR_UNIMPLEMENTED;
+}
+
+int gswa_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
+             const void *w_q, const void *w_k, const void *y, const float *lse, const void *dy,
+             void *dq, void *dk, void *dv, void *dg, float *dw_q, float *dw_k, void *workspace,
+             size_t workspace_bytes, void *stream)
+{
+    (void)s; (void)q; (void)k; (void)v; (void)g; (void)w_q; (void)w_k; (void)y; (void)lse;
+    (void)dy; (void)dq; (void)dk; (void)dv; (void)dg; (void)dw_q; (void)dw_k; (void)workspace;
+    (void)workspace_bytes; (void)stream;
+    return GSWA_ERR_UNIMPLEMENTED;
+}
+
+int full_attn_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
+                  const void *w_q, const void *w_k, const void *y, const float *lse,
+                  const void *dy, void *dq, void *dk, void *dv, float *dw_q, float *dw_k,
+                  void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)y; (void)lse; (void)dy;
+    (void)dq; (void)dk; (void)dv; (void)dw_q; (void)dw_k; (void)workspace;
+    (void)workspace_bytes; (void)stream;
+    return GSWA_ERR_UNIMPLEMENTED;
+}
+
+int gswa_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
+                const void *w_q, const void *w_k, void *k_ring, void *v_ring, const int64_t *pos,
+                void *y, void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)s; (void)q; (void)k; (void)v; (void)g; (void)w_q; (void)w_k; (void)k_ring;
+    (void)v_ring; (void)pos; (void)y; (void)workspace; (void)workspace_bytes; (void)stream;
+    return GSWA_ERR_UNIMPLEMENTED;
+}
+
+int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v,
+                const void *w_q, const void *w_k, void *k_cache, void *v_cache,
+                const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
+                void *stream)
+{
+    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)k_cache; (void)v_cache;
+    (void)pos; (void)y; (void)workspace; (void)workspace_bytes; (void)stream;
+    return GSWA_ERR_UNIMPLEMENTED;
+}
+
+size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
+{
+    (void)op;
+    (void)s;
+    return 0;
+}
+
+int64_t gswa_kv_cache_bytes(int n_global_layers, int n_window_layers, int window, int Hkv, int D,
+                            int bytes_per_elem, int64_t T)
+{
+    if (n_global_layers < 0 || n_window_layers < 0 || window < 0 || Hkv < 0 || D < 0 ||
+        bytes_per_elem < 0 || T < 0)
+        return -1;
+    const int64_t per_token = 2LL * Hkv * D * bytes_per_elem;
+    const int64_t swa_tokens = T < window ? T : window;
+    return per_token * ((int64_t)n_global_layers * T + (int64_t)n_window_layers * swa_tokens);
+}
+
+int gswa_check_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GSWA_ERR_LAUNCH;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, gswa::g_status, sizeof v) != cudaSuccess) return GSWA_ERR_LAUNCH;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(gswa::g_status, &zero, sizeof zero) != cudaSuccess) return GSWA_ERR_LAUNCH;
+        return GSWA_ERR_TIMEOUT;
+    }
+    return GSWA_OK;
+}
+
+const char *gswa_strerror(int code)
+{
+    switch (code) {
+    case GSWA_OK: return "ok";
+    case GSWA_ERR_INVALID_ARG: return "invalid argument";
+    case GSWA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GSWA_ERR_MISALIGNED: return "misaligned pointer";
+    case GSWA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case GSWA_ERR_LAUNCH: return "CUDA launch or runtime error";
+    case GSWA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case GSWA_ERR_UNIMPLEMENTED: return "not implemented";
+    case GSWA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown error";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+/*
+ * gswa.h -- C ABI of the ZGCM-1 attention core on B200 (sm_100a).
+ *
+ * The operation (ZGCM-1, §2.1 Model overview and Figure 3 caption; §2.3
+ * KV-cache analysis; §3.2 Mid-training): for projected queries q, keys k,
+ * values v and gate logits g of one attention layer,
+ *
+ *   q~ = RoPE(RMSNorm(q) * w_q),  k~ = RoPE(RMSNorm(k) * w_k)
+ *        RMSNorm per (token, head) over the head dim, eps inside the root;
+ *        RoPE rotates the first R dims as pairs (p, p + R/2) by the angle
+ *        pos * rope_base^(-2p/R), pos = 0-based token index;
+ *   s_ij = scale * <q~_i, k~_j>, query head h reads KV head h / (Hq/Hkv);
+ *   gated sliding-window layers: key j visible to query i iff i-W < j <= i,
+ *        y_i = softmax_j(s_ij) V  ⊙  sigmoid(g_i)        (GatedSWA core)
+ *   global layers: key j visible iff j <= i, y_i = softmax_j(s_ij) V.
+ * The q/k/v/g projections before and o_proj after are not part of it.
+ *
+ * Conventions shared by every entry point:
+ *   - Layouts are dense row-major: q, g, y, dq, dg, dy: [B, T, Hq, D];
+ *     k, v, dk, dv: [B, T, Hkv, D]; w_q, w_k: [D]; lse: [B, Hq, T].
+ *     Tensors are bf16 unless stated; lse and dw are float32.
+ *   - Pointers marked "device" must point to device memory of the current
+ *     CUDA device; tensor pointers must be 16-byte aligned.
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     device memory, keeps no pointer past the call and frees nothing.
+ *     Workspace, when an operation needs one, is caller-provided and sized
+ *     by gswa_workspace_bytes().
+ *   - Execution: asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are reported synchronously by the
+ *     return value; a device-side wait that gave up (a bounded wait that
+ *     timed out) is reported by gswa_check_status().
+ *   - Supported shapes: D = 128, Hq = 4 * Hkv, 0 <= R <= D and R even,
+ *     1 <= window <= 128 for the sliding-window entry points.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef GSWA_H
+#define GSWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define GSWA_OK 0
+#define GSWA_ERR_INVALID_ARG (-1)       /* null pointer, negative size, bad enum */
+#define GSWA_ERR_UNSUPPORTED_SHAPE (-2) /* D != 128, Hq != 4*Hkv, window out of range ... */
+#define GSWA_ERR_MISALIGNED (-3)        /* a tensor pointer is not 16-byte aligned */
+#define GSWA_ERR_WORKSPACE_TOO_SMALL (-4)
+#define GSWA_ERR_LAUNCH (-5)            /* a CUDA runtime call failed */
+#define GSWA_ERR_TIMEOUT (-6)           /* a bounded device wait gave up */
+#define GSWA_ERR_UNIMPLEMENTED (-7)
+#define GSWA_ERR_NO_DEVICE (-8)         /* no sm_100 device current */
+
+/* Operation ids for gswa_workspace_bytes(). */
+#define GSWA_OP_GSWA_FWD 0
+#define GSWA_OP_FULL_FWD 1
+#define GSWA_OP_GSWA_BWD 2
+#define GSWA_OP_FULL_BWD 3
+#define GSWA_OP_GSWA_DECODE 4
+#define GSWA_OP_FULL_DECODE 5
+
+/* Problem description (plain values, passed by pointer, read during the call only). */
+typedef struct gswa_shape {
+    int32_t B;         /* batch (sequences) */
+    int32_t T;         /* tokens per sequence (prefill/backward); unused by decode */
+    int32_t Hq;        /* query heads (32 in ZGCM-1) */
+    int32_t Hkv;       /* key/value heads (8 in ZGCM-1); Hq = 4 * Hkv */
+    int32_t D;         /* head dim; must be 128 */
+    int32_t window;    /* W of the sliding window (128 in ZGCM-1); ring-cache slots in decode */
+    int32_t rope_dims; /* R rotated dims (42 = 0.33 of 128, rounded to even) */
+    int32_t cache_len; /* decode with a linear cache: capacity Tmax of the cache */
+    double rope_base;  /* 1e4, or 1e7 for the 256K stage (§3.2) */
+    float eps;         /* RMSNorm epsilon (1e-6) */
+    float scale;       /* softmax scale (1/sqrt(D)) */
+} gswa_shape_t;
+
+/*
+ * Gated sliding-window attention forward (§2.1 Figure 3: A_SWA(q,k,v) ⊙ σ(g)).
+ *   q, g [B,T,Hq,D], k, v [B,T,Hkv,D], w_q, w_k [D]: device, bf16, read.
+ *   y [B,T,Hq,D] bf16: device, written (gated output).
+ *   lse [B,Hq,T] f32: device, written (natural-log softmax normaliser of each
+ *     row, for the backward); may be NULL.
+ *   workspace may be NULL (needs 0 bytes).
+ */
+int gswa_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+             const void *g, const void *w_q, const void *w_k, void *y, float *lse,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Full causal attention forward of the 5 global layers (§2.1: global
+ * layers attend over the whole context and drop the gate).  Same layouts
+ * as gswa_fwd without g; shape->window is ignored.
+ */
+int full_attn_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+                  const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
+/*
+ * Backward of gswa_fwd.  Reads q, k, v, g, w_q, w_k, the forward's y and lse,
+ * and the upstream gradient dy [B,T,Hq,D]; writes dq, dg [B,T,Hq,D],
+ * dk, dv [B,T,Hkv,D] (bf16) and dw_q, dw_k [D] (f32).  All device.
+ */
+int gswa_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+             const void *g, const void *w_q, const void *w_k, const void *y, const float *lse,
+             const void *dy, void *dq, void *dk, void *dv, void *dg, float *dw_q, float *dw_k,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Backward of full_attn_fwd (no gate, no dg). */
+int full_attn_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+                  const void *w_q, const void *w_k, const void *y, const float *lse,
+                  const void *dy, void *dq, void *dk, void *dv, float *dw_q, float *dw_k,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step of a gated sliding-window layer over a ring KV cache
+ * (§2.3: the SWA layers keep a fixed window of W tokens in the cache).
+ *   q, g [B,Hq,D], k, v [B,Hkv,D]: the new token's projections (device, bf16).
+ *   k_ring, v_ring [B,Hkv,W,D] bf16 (device, read and written): the token at
+ *     position t lives in slot t mod W; k_ring holds normed+rotated keys,
+ *     v_ring raw values.  The new token is written to slot pos mod W and is
+ *     part of its own window; slots holding positions < 0 are ignored.
+ *   pos [B] int64 (device): position of the new token of each sequence.
+ *   y [B,Hq,D] bf16 (device, written).  shape->window = W = ring slots.
+ */
+int gswa_decode(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+                const void *g, const void *w_q, const void *w_k, void *k_ring, void *v_ring,
+                const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
+                void *stream);
+
+/*
+ * One decode step of a global layer over a linear cache [B,Hkv,Tmax,D]
+ * (Tmax = shape->cache_len): writes the new key/value at row pos and attends
+ * over rows 0..pos.  Split over the cache length; needs a workspace.
+ */
+int full_decode(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+                const void *w_q, const void *w_k, void *k_cache, void *v_cache,
+                const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
+                void *stream);
+
+/* Workspace bytes an operation needs for `shape` (0 when none). */
+size_t gswa_workspace_bytes(int op, const gswa_shape_t *shape);
+
+/*
+ * KV-cache bytes of a layer stack at context length T (§2.3): every cached
+ * token costs 2 * Hkv * D * bytes_per_elem bytes per layer; a global layer
+ * caches all T tokens, a sliding-window layer min(T, window).  Host only.
+ * Returns -1 on a negative argument.
+ */
+int64_t gswa_kv_cache_bytes(int n_global_layers, int n_window_layers, int window, int Hkv,
+                            int D, int bytes_per_elem, int64_t T);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device: GSWA_OK, GSWA_ERR_TIMEOUT if a bounded wait inside a
+ * kernel gave up since the last check, or GSWA_ERR_LAUNCH on a CUDA error.
+ */
+int gswa_check_status(void *stream);
+
+/* Human-readable name of a return code (static string). */
+const char *gswa_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSWA_H */

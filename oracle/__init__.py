@@ -87,6 +87,20 @@ def _ptr(a) -> int | None:
     return None if a is None else a.ctypes.data
 
 
+class _Keep:
+    """Holds every converted input array until the C call has returned (a
+    pointer to a temporary copy would otherwise dangle)."""
+
+    def __init__(self, f64: bool):
+        self.f64 = f64
+        self.arrays = []
+
+    def __call__(self, t):
+        a = _arr(t, self.f64)
+        self.arrays.append(a)
+        return _ptr(a)
+
+
 def _check(rc: int, what: str):
     if rc != 0:
         raise RuntimeError(f"oracle {what} failed with code {rc}")
@@ -103,11 +117,11 @@ def qk_prep(x, w, rope_dims, rope_base, eps, pos0=0, L=None):
     read as float64)."""
     L = L or lib()
     f64 = _is_f64(x)
-    xa, wa = _arr(x, f64), _arr(w, f64)
-    B, T, H, D = xa.shape
+    keep = _Keep(f64)
+    B, T, H, D = x.shape
     out = np.empty((B, T, H, D), np.float64)
     _check(L.oracle_qk_prep(int(f64), B, T, H, D, rope_dims, rope_base, eps, pos0,
-                            _ptr(xa), _ptr(wa), _ptr(out)), "qk_prep")
+                            keep(x), keep(w), _ptr(out)), "qk_prep")
     return out
 
 
@@ -120,10 +134,9 @@ def attn_fwd(q, k, v, g, wq, wk, *, window, gated, rope_dims, rope_base, eps, sc
     """
     L = L or lib()
     f64 = _is_f64(q)
-    qa, ka, va = _arr(q, f64), _arr(k, f64), _arr(v, f64)
-    ga = _arr(g, f64) if gated else None
-    B, T, Hq, D = qa.shape
-    Hkv = ka.shape[2]
+    keep = _Keep(f64)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
     rows_np = None
     nrows = T
     if rows is not None:
@@ -132,8 +145,8 @@ def attn_fwd(q, k, v, g, wq, wk, *, window, gated, rope_dims, rope_base, eps, sc
     y = np.empty((B, nrows, Hq, D), np.float64)
     lse = np.empty((B, Hq, nrows), np.float64)
     _check(L.oracle_attn_fwd(int(f64), B, T, Hq, Hkv, D, window, int(bool(gated)), rope_dims,
-                             rope_base, eps, scale, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ga),
-                             _ptr(_arr(wq, f64)), _ptr(_arr(wk, f64)), nrows, _ptr(rows_np),
+                             rope_base, eps, scale, keep(q), keep(k), keep(v),
+                             keep(g) if gated else None, keep(wq), keep(wk), nrows, _ptr(rows_np),
                              _ptr(y), _ptr(lse)), "attn_fwd")
     return y, lse
 
@@ -143,10 +156,9 @@ def attn_bwd(q, k, v, g, wq, wk, dy, *, window, gated, rope_dims, rope_base, eps
     """Gradients (dq, dk, dv, dg or None, dwq, dwk) in float64."""
     L = L or lib()
     f64 = _is_f64(q)
-    qa, ka, va, dya = _arr(q, f64), _arr(k, f64), _arr(v, f64), _arr(dy, f64)
-    ga = _arr(g, f64) if gated else None
-    B, T, Hq, D = qa.shape
-    Hkv = ka.shape[2]
+    keep = _Keep(f64)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
     dq = np.empty((B, T, Hq, D), np.float64)
     dk = np.empty((B, T, Hkv, D), np.float64)
     dv = np.empty((B, T, Hkv, D), np.float64)
@@ -154,8 +166,8 @@ def attn_bwd(q, k, v, g, wq, wk, dy, *, window, gated, rope_dims, rope_base, eps
     dwq = np.empty(D, np.float64)
     dwk = np.empty(D, np.float64)
     _check(L.oracle_attn_bwd(int(f64), B, T, Hq, Hkv, D, window, int(bool(gated)), rope_dims,
-                             rope_base, eps, scale, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ga),
-                             _ptr(_arr(wq, f64)), _ptr(_arr(wk, f64)), _ptr(dya), _ptr(dq),
+                             rope_base, eps, scale, keep(q), keep(k), keep(v),
+                             keep(g) if gated else None, keep(wq), keep(wk), keep(dy), _ptr(dq),
                              _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq), _ptr(dwk)), "attn_bwd")
     return dq, dk, dv, dg, dwq, dwk
 
@@ -166,19 +178,17 @@ def decode(q, k, v, g, wq, wk, k_cache, v_cache, pos, *, window, gated, rope_dim
     cache [B, Hkv, Tmax, D].  Returns (y [B, Hq, D], k_new_prepared [B, Hkv, D])."""
     L = L or lib()
     f64 = _is_f64(q)
-    qa, ka, va = _arr(q, f64), _arr(k, f64), _arr(v, f64)
-    ga = _arr(g, f64) if gated else None
-    kc, vc = _arr(k_cache, f64), _arr(v_cache, f64)
-    B, Hq, D = qa.shape
-    Hkv = ka.shape[1]
-    Tmax = kc.shape[2]
+    keep = _Keep(f64)
+    B, Hq, D = q.shape
+    Hkv = k.shape[1]
+    Tmax = k_cache.shape[2]
     pos_np = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(B))
     y = np.empty((B, Hq, D), np.float64)
     kp = np.empty((B, Hkv, D), np.float64)
     _check(L.oracle_decode(int(f64), B, Hq, Hkv, D, window, int(bool(gated)), rope_dims,
-                           rope_base, eps, scale, Tmax, _ptr(pos_np), _ptr(qa), _ptr(ka),
-                           _ptr(va), _ptr(ga), _ptr(_arr(wq, f64)), _ptr(_arr(wk, f64)),
-                           _ptr(kc), _ptr(vc), _ptr(y), _ptr(kp)), "decode")
+                           rope_base, eps, scale, Tmax, _ptr(pos_np), keep(q), keep(k),
+                           keep(v), keep(g) if gated else None, keep(wq), keep(wk),
+                           keep(k_cache), keep(v_cache), _ptr(y), _ptr(kp)), "decode")
     return y, kp
 
 

@@ -1,0 +1,76 @@
+"""The C ABI library: builds, loads without a GPU, exports every declared symbol,
+and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import global_causal_attention_b200 as gca
+from global_causal_attention_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gca.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10, names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+
+
+def test_strerror(L):
+    assert gca.strerror(0) == "ok"
+    assert "timed out" in gca.strerror(-6)
+
+
+def test_kv_cache_bytes_matches_pages():
+    # ZGCM-1 §2.3: 4 KiB per token per layer, 128 KiB all-global, 32.0 / 5.0 GiB at 256K
+    assert gca.gswa_kv_cache_bytes(1, 0, 128, 8, 128, 2, 1) == 4096
+    assert gca.gswa_kv_cache_bytes(32, 0, 128, 8, 128, 2, 1) == 128 * 1024
+    assert gca.gswa_kv_cache_bytes(32, 0, 128, 8, 128, 2, 262144) == 32 * 2**30
+    hyb = gca.gswa_kv_cache_bytes(5, 27, 128, 8, 128, 2, 262144)
+    assert abs(hyb / 2**30 - 5.0) < 0.05
+    assert gca.gswa_kv_cache_bytes(-1, 0, 128, 8, 128, 2, 1) == -1
+
+
+def _call_fwd(L, s, ptr=16):
+    return L.gswa_fwd(ctypes.byref(s), ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, None, 0, None)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("D", 64, -2), ("Hq", 6, -2), ("window", 0, -2), ("window", 129, -2), ("rope_dims", 43, -2),
+    ("rope_dims", 130, -2), ("B", -1, -1), ("eps", -1.0, -1),
+])
+def test_host_validation(L, field, value, code):
+    s = gca.make_shape(1, 64, 4, 1)
+    setattr(s, field, value)
+    assert _call_fwd(L, s) == code
+
+
+def test_null_and_misaligned_pointers(L):
+    s = gca.make_shape(1, 64, 4, 1)
+    assert L.gswa_fwd(None, 16, 16, 16, 16, 16, 16, 16, None, None, 0, None) == -1
+    assert L.gswa_fwd(ctypes.byref(s), None, 16, 16, 16, 16, 16, 16, None, None, 0, None) == -1
+    assert _call_fwd(L, s, ptr=18) == -3
+
+
+def test_empty_problem_is_a_no_op(L):
+    s = gca.make_shape(0, 64, 4, 1)
+    assert _call_fwd(L, s, ptr=0) == 0

@@ -1,0 +1,67 @@
+"""Parity of the CUDA gated-SWA forward with the float64 oracle (needs a B200)."""
+import pytest
+import torch
+
+import global_causal_attention_b200 as gca
+import oracle
+from tests.parity import assert_fwd_close
+from workloads import WORKLOADS, Shape, attention_inputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # name: (shape, seed, random_weights)
+    "tiny_512": (WORKLOADS["tiny"], 0, False),
+    "ragged_200_gqa2": (Shape(B=2, T=200, Hq=8, Hkv=2), 1, True),
+    "ragged_37_w16": (Shape(B=1, T=37, Hq=4, Hkv=1, window=16), 2, True),
+    "single_token": (Shape(B=3, T=1, Hq=4, Hkv=1), 3, False),
+    "window_1": (Shape(B=2, T=100, Hq=4, Hkv=1, window=1), 4, True),
+    "window_64_T161": (Shape(B=1, T=161, Hq=8, Hkv=2, window=64), 5, False),
+    "rope_0": (Shape(B=1, T=300, Hq=4, Hkv=1, rope_dims=0), 6, False),
+    "rope_128": (Shape(B=1, T=300, Hq=4, Hkv=1, rope_dims=128), 7, True),
+    "base_1e7_T1000": (Shape(B=1, T=1000, Hq=8, Hkv=2, rope_base=1e7), 8, False),
+    "many_strips_T96": (Shape(B=5, T=96, Hq=12, Hkv=3), 9, True),
+}
+
+
+def run_gpu(s, x):
+    xd = {n: t.cuda() for n, t in x.items()}
+    y, lse = gca.gswa_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["wq"], xd["wk"], window=s.window,
+                          rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    assert gca.gswa_check_status() == 0
+    return y, lse
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_swa_fwd_matches_oracle(name):
+    s, seed, rw = CASES[name]
+    x = attention_inputs(s, seed, random_weights=rw)
+    y, lse = run_gpu(s, x)
+    yo, lo = oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
+                             gated=True, **oracle.shape_kwargs(s))
+    assert_fwd_close(y, yo, "y")
+    assert_fwd_close(lse, lo, "lse")
+
+
+def test_swa_fwd_deterministic():
+    s = Shape(B=2, T=257, Hq=8, Hkv=2)
+    x = attention_inputs(s, 11)
+    y1, l1 = run_gpu(s, x)
+    y2, l2 = run_gpu(s, x)
+    assert torch.equal(y1, y2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("workload,nrows", [("train_4k", 48), ("prefill_64k", 24), ("prefill_256k", 16)])
+def test_swa_fwd_full_size_sampled_rows(workload, nrows):
+    """The full workload in the launch configuration the benchmark times; the oracle
+    evaluates a seeded sample of query rows (all heads, all sequences)."""
+    s = WORKLOADS[workload]
+    x = attention_inputs(s, 0, device="cuda")
+    y, lse = gca.gswa_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
+                          rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    assert gca.gswa_check_status() == 0
+    rows = sample_rows(s.T, nrows, seed=1)
+    yo, lo = oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
+                             gated=True, rows=rows.numpy(), **oracle.shape_kwargs(s))
+    assert_fwd_close(y[:, rows.cuda()], yo, "y")
+    assert_fwd_close(lse[:, :, rows.cuda()], lo, "lse")
