@@ -34,6 +34,16 @@ std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
+template <typename K>
+bool set_smem(K kernel, uint32_t bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+           cudaSuccess;
+}
+
+// Rotated dims the kernels are compiled for (the row is held in registers).
+bool rope_dims_supported(int R) { return R == 0 || R == 42 || R == 64 || R == 128; }
+
 // Per-device set-up (compute capability check, kernel attributes, SM count),
 // done once per device under a lock.
 int device_setup(int *num_sms)
@@ -52,9 +62,10 @@ int device_setup(int *num_sms)
             d.status = GSWA_ERR_NO_DEVICE;
         } else if (major != 10 || minor != 0) {
             d.status = GSWA_ERR_NO_DEVICE;  // built for sm_100a only
-        } else if (cudaFuncSetAttribute(gswa::swa::swa_fwd_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)gswa::swa::kSmemBytes) != cudaSuccess) {
+        } else if (set_smem(gswa::swa::swa_fwd_kernel<0>, gswa::swa::kSmemBytes) ||
+                   set_smem(gswa::swa::swa_fwd_kernel<42>, gswa::swa::kSmemBytes) ||
+                   set_smem(gswa::swa::swa_fwd_kernel<64>, gswa::swa::kSmemBytes) ||
+                   set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes)) {
             d.status = GSWA_ERR_LAUNCH;
         }
         if (d.status == GSWA_OK && g_encode == nullptr) {
@@ -121,6 +132,7 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
     int rc = check_common(s);
     if (rc != GSWA_OK) return rc;
     if (s->window < 1 || s->window > 128) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (!rope_dims_supported(s->rope_dims)) return GSWA_ERR_UNSUPPORTED_SHAPE;
     if ((long long)s->B * s->T == 0) return GSWA_OK;
     if (!q || !k || !v || !g || !w_q || !w_k || !y) return GSWA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(y) ||
@@ -145,7 +157,6 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
     p.Hq = s->Hq;
     p.Hkv = s->Hkv;
     p.window = s->window;
-    p.R = s->rope_dims;
     p.nsteps = (s->T + gswa::swa::kTok - 1) / gswa::swa::kTok;
     p.units = (long long)s->B * s->Hkv * p.nsteps;
     p.eps = s->eps;
@@ -156,8 +167,15 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
     fill_theta(p.theta, s->rope_dims, s->rope_base);
 
     const long long grid = p.units < num_sms ? p.units : num_sms;
-    gswa::swa::swa_fwd_kernel<<<(unsigned)grid, gswa::swa::kThreads, gswa::swa::kSmemBytes,
-                                static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tg, ty, p);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 gr((unsigned)grid), bl(gswa::swa::kThreads);
+    const uint32_t sm = gswa::swa::kSmemBytes;
+    switch (s->rope_dims) {
+    case 0: gswa::swa::swa_fwd_kernel<0><<<gr, bl, sm, st>>>(tq, tk, tv, tg, ty, p); break;
+    case 42: gswa::swa::swa_fwd_kernel<42><<<gr, bl, sm, st>>>(tq, tk, tv, tg, ty, p); break;
+    case 64: gswa::swa::swa_fwd_kernel<64><<<gr, bl, sm, st>>>(tq, tk, tv, tg, ty, p); break;
+    default: gswa::swa::swa_fwd_kernel<128><<<gr, bl, sm, st>>>(tq, tk, tv, tg, ty, p); break;
+    }
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 

@@ -10,25 +10,34 @@
 // Work unit: a 32-token query block of one (sequence, KV head) pair, i.e. the
 // 4 query heads of a GQA group packed as M = 128 tensor-core rows
 // (row r = 4 * token + head-in-group).  Its keys are the 160 keys
-// [i0 - 128, i0 + 32): five 32-key blocks.  Persistent CTAs walk consecutive
-// blocks of a strip, so each K/V block is fetched from HBM once and kept in
-// a six-slot shared-memory ring while the window slides over it.
+// [i0 - 128, i0 + 32): five 32-key blocks, so one QK^T MMA of N = 160 covers
+// every key any of its rows can see and the softmax needs a single pass (no
+// running rescale).  Persistent CTAs walk consecutive blocks of a strip, so
+// each K/V block is fetched from HBM once and kept in a six-slot shared-memory
+// ring while the window slides over it.
 //
 // Warp roles (16 warps):
-//   warp 0      TMA producer: Q, g tiles (2 stages) and K/V blocks (ring)
-//   warp 1      TMEM owner and tcgen05.mma issuer
+//   warp 0      TMA producer of K/V blocks (ring)
+//   warp 1      TMEM owner and tcgen05.mma issuer; it polls S-, PV- and
+//               Q-slot readiness independently (so none waits behind another)
+//               and also issues the TMA loads of the Q tiles (2 stages)
 //   warp 2      key prologue: RMSNorm + RoPE of each new K block, in place
 //   warp 3      idle
 //   warps 4-7   query prologue: RMSNorm + RoPE of the 128 Q rows, in place
-//   warps 8-11  softmax: S (TMEM) -> P (bf16, TMEM), row max/sum, lse
-//   warps 12-15 epilogue: O (TMEM) / l ⊙ σ(g) -> y, TMA store
+//   warps 8-11  softmax: S (TMEM) -> P (bf16, TMEM), 1/l (TMEM), lse
+//   warps 12-15 epilogue: σ(g) into the gate tile ahead of time, then
+//               O (TMEM) * 1/l * σ -> y in the gate tile, TMA store; its thread 0
+//               also loads the gate tiles (2 stages), reusing each slot as soon
+//               as the y store has read it
 //
 // TMEM (512 columns) holds two buffers of 256 columns: S at +0 (160 f32
-// columns), P at +0 (80 columns of bf16 pairs, written over S once read)
-// and O at +128 (128 f32 columns, written only after P is complete).
+// columns), P at +0 (80 columns of bf16 pairs, written over S once read),
+// 1/l at +80, and O at +128 (128 f32 columns, written only after P is done).
 #pragma once
 
 #include <cuda.h>
+
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -36,12 +45,13 @@ namespace gswa {
 namespace swa {
 
 constexpr int kD = 128;
-constexpr int kTok = 32;                 // query tokens per unit
-constexpr int kRows = 128;               // MMA M
-constexpr int kSpanBlocks = 5;           // 160-key window span in 32-key blocks
-constexpr int kRing = 6;                 // K/V ring slots
+constexpr int kTok = 32;                  // query tokens per unit
+constexpr int kRows = 128;                // MMA M
+constexpr int kSpanBlocks = 5;            // 160-key window span in 32-key blocks
+constexpr int kRing = 6;                  // K/V ring slots
 constexpr int kSpan = kSpanBlocks * kTok; // 160
 constexpr int kThreads = 512;
+constexpr int kColInvL = 80;              // TMEM column of 1/l inside a buffer
 
 // Shared-memory map (offsets from a 1024-byte-aligned base).
 constexpr uint32_t kHalfRowBytes = 128;                       // 64 bf16 per swizzled row
@@ -53,10 +63,9 @@ constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + 2 * kRingHalfBytes;        // 49152
 constexpr uint32_t kOffQ = kOffV + 2 * kRingHalfBytes;        // 98304
 constexpr uint32_t kOffG = kOffQ + 2 * kTileBytes;            // 163840
-constexpr uint32_t kOffWq = kOffG + 2 * kTileBytes;           // 229376 (bf16[128])
-constexpr uint32_t kOffWk = kOffWq + 256;
-constexpr uint32_t kOffInvL = kOffWk + 256;                   // f32[2][128]
-constexpr uint32_t kOffBar = kOffInvL + 2 * kRows * 4;
+constexpr uint32_t kOffWq = kOffG + 2 * kTileBytes;           // 229376 (f32[128])
+constexpr uint32_t kOffWk = kOffWq + 512;                     // f32[128]
+constexpr uint32_t kOffBar = kOffWk + 512;
 constexpr int kNumBars = 33;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -72,7 +81,7 @@ enum : int {
 };
 
 struct Params {
-    int B, T, Hq, Hkv, window, R;
+    int B, T, Hq, Hkv, window;
     int nsteps;        // ceil(T / 32)
     long long units;   // B * Hkv * nsteps
     float eps;
@@ -82,22 +91,32 @@ struct Params {
     double theta[64];  // rope_base^(-2p/R), p < R/2
 };
 
-struct Unit {
+// Walks the units [u0, u1) of a CTA in order: (sequence b, kv head, step s).
+struct Walker {
     int b, kvh, s;
-    bool first, last;
+    __device__ __forceinline__ void init(const Params &p, long long u0)
+    {
+        const long long strip = u0 / p.nsteps;
+        s = (int)(u0 - strip * p.nsteps);
+        b = (int)(strip / p.Hkv);
+        kvh = (int)(strip - (long long)b * p.Hkv);
+    }
+    __device__ __forceinline__ void next(const Params &p)
+    {
+        if (++s == p.nsteps) {
+            s = 0;
+            if (++kvh == p.Hkv) {
+                kvh = 0;
+                ++b;
+            }
+        }
+    }
+    __device__ __forceinline__ bool first(int idx) const { return idx == 0 || s == 0; }
+    __device__ __forceinline__ bool last(const Params &p, int idx, int n) const
+    {
+        return idx == n - 1 || s == p.nsteps - 1;
+    }
 };
-
-__device__ __forceinline__ Unit unit_of(const Params &p, long long u, long long u0, long long u1)
-{
-    Unit x;
-    long long strip = u / p.nsteps;
-    x.s = (int)(u - strip * p.nsteps);
-    x.b = (int)(strip / p.Hkv);
-    x.kvh = (int)(strip - (long long)x.b * p.Hkv);
-    x.first = (u == u0) || (x.s == 0);
-    x.last = (u == u1 - 1) || (x.s == p.nsteps - 1);
-    return x;
-}
 
 __device__ __forceinline__ int ring_slot(int kb) { return ((kb % kRing) + kRing) % kRing; }
 
@@ -109,102 +128,242 @@ __device__ __forceinline__ uint32_t chunk_off(int r, int c, uint32_t half_stride
            ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
 
-// Byte offset of element d of row r (same layout).
-__device__ __forceinline__ uint32_t elem_off(int r, int d, uint32_t half_stride)
-{
-    return chunk_off(r, d >> 3, half_stride) + (uint32_t)(d & 7) * 2;
-}
-
-// cos/sin of the rotary angle pos * theta, reduced in double precision first
-// so that positions up to 2^18 keep full single-precision accuracy.
+// cos/sin of the rotary angle pos * theta, reduced modulo 2π in double
+// precision first so that positions up to 2^18 keep full accuracy.
 __device__ __forceinline__ void rope_cs(double theta, int pos, float &c, float &s)
 {
     const double two_pi = 6.283185307179586;
-    double phi = (double)pos * theta;
-    double k = rint(phi * (1.0 / two_pi));
-    float r = (float)fma(-k, two_pi, phi);
-    sincosf(r, &s, &c);
+    const double phi = (double)pos * theta;
+    const double k = rint(phi * (1.0 / two_pi));
+    const float r = (float)fma(-k, two_pi, phi);
+    // |r| <= pi here, where the hardware sine/cosine are accurate to ~2^-21.
+    __sincosf(r, &s, &c);
 }
 
-// RMSNorm then partial RoPE of one head row held in shared memory (bf16,
-// swizzled), in place, one thread per row.  Dims >= R are scaled only; the
-// rotated pairs (p, p + R/2) are normalised and rotated in f32 and rounded
-// once.  `cs_from_group` lets 4 neighbouring lanes that share a token split
-// the cos/sin evaluations (each computes every 4th pair, then they swap).
-template <bool kShareInQuad>
-__device__ __forceinline__ void prep_row_smem(uint8_t *tile, uint32_t half_stride, int row,
-                                              const __nv_bfloat16 *w, int R, float eps, int pos,
-                                              const double *theta)
-{
-    // pass 1: mean square of the raw row
-    float ss = 0.f;
+// cos/sin of the rotary angles of one thread's token, by angle addition:
+// the angle (i0 + t) theta_p of token t of a 32-token block starting at i0 is
+// split into a block part i0 theta_p, evaluated once per block (lane p of the
+// warp evaluates pair p and the warp shares it by shuffle), and a row part
+// t theta_p, evaluated once per kernel (t is fixed per thread).  Then
+// cos = cA cB - sA sB and sin = sA cB + cA sB cost four FMAs per pair.
+// kStride/kOffset select the pairs this thread owns (p = kOffset + k kStride).
+template <int H, int kStride>
+struct RopeTab {
+    static constexpr int kN = (H + kStride - 1) / kStride;
+    float cb[kN > 0 ? kN : 1], sb[kN > 0 ? kN : 1];  // row part of the owned pairs
+    float ca, sa, ca2, sa2;                           // block part of pairs lane, lane + 32
+    __device__ __forceinline__ void init_rows(int t, int offset, const double *theta)
+    {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        uint4 v = *reinterpret_cast<const uint4 *>(tile + chunk_off(row, c, half_stride));
-        uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16(u[e]);
-            ss = fmaf(f.x, f.x, ss);
-            ss = fmaf(f.y, f.y, ss);
+        for (int k = 0; k < kN; ++k) {
+            const int pp = offset + k * kStride;
+            cb[k] = 1.f;
+            sb[k] = 0.f;
+            if (pp < H) rope_cs(theta[pp], t, cb[k], sb[k]);
         }
     }
-    const float r = rsqrtf(ss * (1.0f / kD) + eps);
-    // pass 2: plain scaling of the dims past the rotated slice
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const int d0 = c * 8;
-        if (d0 + 8 <= R) continue;
-        uint4 *ptr = reinterpret_cast<uint4 *>(tile + chunk_off(row, c, half_stride));
-        uint4 v = *ptr;
-        uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16(u[e]);
-            const int d = d0 + 2 * e;
-            float a = (d >= R) ? f.x * r * __bfloat162float(w[d]) : f.x;
-            float b = (d + 1 >= R) ? f.y * r * __bfloat162float(w[d + 1]) : f.y;
-            // dims below R keep their raw bits for pass 3
-            u[e] = (d >= R) ? pack_bf16(a, b)
-                            : ((d + 1 >= R) ? ((u[e] & 0xFFFFu) | (pack_bf16(a, b) & 0xFFFF0000u))
-                                            : u[e]);
-        }
-        *ptr = make_uint4(u[0], u[1], u[2], u[3]);
-    }
-    // pass 3: rotate the pairs (p, p + R/2)
-    const int half = R >> 1;
-    if (kShareInQuad) {
+    __device__ __forceinline__ void set_block(int i0, const double *theta)
+    {
         const int lane = threadIdx.x & 31;
-        const int q = lane & 3;
-        for (int p0 = 0; p0 < half; p0 += 4) {
+        ca = ca2 = 1.f;
+        sa = sa2 = 0.f;
+        if (lane < H) rope_cs(theta[lane], i0, ca, sa);
+        if (H > 32 && lane + 32 < H) rope_cs(theta[lane + 32], i0, ca2, sa2);
+    }
+    // cos/sin of owned pair k (pair index pp, a warp-uniform function of k
+    // only when kStride == 1; otherwise each lane passes its own pp)
+    __device__ __forceinline__ void get(int k, int pp, float &c, float &sn) const
+    {
+        const float a_c = __shfl_sync(0xffffffffu, (pp < 32) ? ca : ca2, pp & 31);
+        const float a_s = __shfl_sync(0xffffffffu, (pp < 32) ? sa : sa2, pp & 31);
+        c = a_c * cb[k] - a_s * sb[k];
+        sn = a_s * cb[k] + a_c * sb[k];
+    }
+};
+
+// Same interface as RopeTab for wide rotations (one lane per key row): each
+// cos/sin is evaluated directly, keeping no per-pair registers.
+template <int H>
+struct RopeDirect {
+    int pos0 = 0, t = 0;
+    const double *theta = nullptr;
+    __device__ __forceinline__ void init_rows(int row, int, const double *th)
+    {
+        t = row;
+        theta = th;
+    }
+    __device__ __forceinline__ void set_block(int i0, const double *) { pos0 = i0; }
+    __device__ __forceinline__ void get(int, int pp, float &c, float &sn) const
+    {
+        rope_cs(theta[pp], pos0 + t, c, sn);
+    }
+};
+
+// RMSNorm then partial RoPE of one head row held in shared memory (bf16,
+// swizzled), in place, one thread per row.
+//   r = (mean_d x_d^2 + eps)^-1/2;  u_d = x_d r w_d;
+//   (u_p, u_{p+R/2}) <- (u_p c - u_{p+R/2} s, u_{p+R/2} c + u_p s),  p < R/2
+// computed in f32 and rounded to bf16 once.  The row streams through
+// registers 16 bytes at a time; only the chunks taking part in the rotation
+// are held together.  `tile` is the shared-memory address of the tile, `hs`
+// the byte distance between its two 64-dim halves, `w` the f32 weights
+// (16-byte aligned).  kQuad: the 4 lanes of a quad hold 4 heads of one token;
+// lane q evaluates the cos/sin of pairs p = q mod 4 and the quad swaps them.
+template <int R, bool kQuad, class Tab>
+__device__ __forceinline__ void prep_row(uint32_t tile, uint32_t hs, int row, const float *w, float eps,
+                                         const Tab &tab)
+{
+    constexpr int H = R / 2;
+    constexpr bool kAligned = (H % 8) == 0;
+    constexpr int kRot = (R + 7) / 8;      // leading chunks holding a rotated dim
+    constexpr int kPair = kAligned ? H / 8 : 0;  // aligned: chunk c pairs with chunk c + kPair
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    const int lane = threadIdx.x & 31;
+    // pass 1: mean square of the raw row (eight independent accumulators)
+    float ss[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = lds128(tile + chunk_off(row, c, hs));
+        const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16(u4[e]);
+            ss[2 * e] = fmaf(f.x, f.x, ss[2 * e]);
+            ss[2 * e + 1] = fmaf(f.y, f.y, ss[2 * e + 1]);
+        }
+    }
+    const float r = rsqrtf(((ss[0] + ss[1]) + (ss[2] + ss[3]) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) *
+                               (1.0f / kD) + eps);
+    // scaled values of one chunk
+    auto scale8 = [&](const uint4 v, int c, float (&u)[8]) {
+        const float4 wa = w4[2 * c], wb = w4[2 * c + 1];
+        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16(u4[e]);
+            u[2 * e] = f.x * (r * wv[2 * e]);
+            u[2 * e + 1] = f.y * (r * wv[2 * e + 1]);
+        }
+    };
+    auto pack8 = [](const float *u) {
+        return make_uint4(pack_bf16(u[0], u[1]), pack_bf16(u[2], u[3]), pack_bf16(u[4], u[5]),
+                          pack_bf16(u[6], u[7]));
+    };
+    // cos/sin of pair p0 + j: from the table (this lane owns p0 + j) or, in quad
+    // mode, from the lane of the quad that owns it
+    auto cs_round = [&](int p0, float &cm, float &sm) {  // quad mode: own pair p0 + (lane & 3)
+        cm = 1.f;
+        sm = 0.f;
+        const int pp = p0 + (lane & 3);
+        tab.get(p0 >> 2, pp < H ? pp : 0, cm, sm);
+    };
+    auto cs_get = [&](int p0, int j, float cm, float sm, float &cc, float &sn) {
+        if constexpr (kQuad) {
+            cc = __shfl_sync(0xffffffffu, cm, (lane & ~3) | j);
+            sn = __shfl_sync(0xffffffffu, sm, (lane & ~3) | j);
+        } else {
+            tab.get(p0 + j, p0 + j, cc, sn);
+        }
+    };
+    // pass 2: chunks without a rotated dim, the next chunk's load ahead of this store
+    constexpr int kPlain0 = kRot;
+    if constexpr (kPlain0 < 16) {
+        uint4 cur = lds128(tile + chunk_off(row, kPlain0, hs));
+#pragma unroll 2
+        for (int c = kPlain0; c < 16; ++c) {
+            uint4 nxt = cur;
+            if (c + 1 < 16) nxt = lds128(tile + chunk_off(row, c + 1, hs));
+            float u[8];
+            scale8(cur, c, u);
+            sts128(tile + chunk_off(row, c, hs), pack8(u));
+            cur = nxt;
+        }
+    }
+    if constexpr (R > 0 && kAligned) {
+        // pairs (p, p + H), H a multiple of 8: chunk c pairs with chunk c + H/8
+#pragma unroll
+        for (int c = 0; c < kPair; ++c) {
+            const uint32_t a1 = tile + chunk_off(row, c, hs);
+            const uint32_t a2 = tile + chunk_off(row, c + kPair, hs);
+            float u1[8], u2[8];
+            scale8(lds128(a1), c, u1);
+            scale8(lds128(a2), c + kPair, u2);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int p0 = 8 * c + 4 * half;
+                float cm = 1.f, sm = 0.f;
+                if constexpr (kQuad) cs_round(p0, cm, sm);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float cc, sn;
+                    cs_get(p0, j, cm, sm, cc, sn);
+                    const int e = 4 * half + j;
+                    const float x1 = u1[e], x2 = u2[e];
+                    u1[e] = x1 * cc - x2 * sn;
+                    u2[e] = x2 * cc + x1 * sn;
+                }
+            }
+            sts128(a1, pack8(u1));
+            sts128(a2, pack8(u2));
+        }
+    } else if constexpr (R > 0) {
+        // general H: hold the kRot leading chunks (<= 48 dims) as floats
+        static_assert(R <= 48, "unaligned rotary widths are held in registers");
+        float u[8 * kRot];
+#pragma unroll
+        for (int c = 0; c < kRot; ++c) {
+            float t8[8];
+            scale8(lds128(tile + chunk_off(row, c, hs)), c, t8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) u[8 * c + e] = t8[e];
+        }
+#pragma unroll
+        for (int p0 = 0; p0 < H; p0 += 4) {
             float cm = 1.f, sm = 0.f;
-            if (p0 + q < half) rope_cs(theta[p0 + q], pos, cm, sm);
+            if constexpr (kQuad) cs_round(p0, cm, sm);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const float c = __shfl_sync(0xffffffffu, cm, (lane & ~3) | j);
-                const float s = __shfl_sync(0xffffffffu, sm, (lane & ~3) | j);
-                const int pp = p0 + j;
-                if (pp < half) {
-                    __nv_bfloat16 *x1 = reinterpret_cast<__nv_bfloat16 *>(tile + elem_off(row, pp, half_stride));
-                    __nv_bfloat16 *x2 = reinterpret_cast<__nv_bfloat16 *>(tile + elem_off(row, pp + half, half_stride));
-                    const float n1 = __bfloat162float(*x1) * r * __bfloat162float(w[pp]);
-                    const float n2 = __bfloat162float(*x2) * r * __bfloat162float(w[pp + half]);
-                    *x1 = __float2bfloat16_rn(n1 * c - n2 * s);
-                    *x2 = __float2bfloat16_rn(n2 * c + n1 * s);
+                if (p0 + j < H) {
+                    float cc, sn;
+                    cs_get(p0, j, cm, sm, cc, sn);
+                    const float x1 = u[p0 + j], x2 = u[p0 + j + H];
+                    u[p0 + j] = x1 * cc - x2 * sn;
+                    u[p0 + j + H] = x2 * cc + x1 * sn;
                 }
             }
         }
-    } else {
-        for (int pp = 0; pp < half; ++pp) {
-            float c, s;
-            rope_cs(theta[pp], pos, c, s);
-            __nv_bfloat16 *x1 = reinterpret_cast<__nv_bfloat16 *>(tile + elem_off(row, pp, half_stride));
-            __nv_bfloat16 *x2 = reinterpret_cast<__nv_bfloat16 *>(tile + elem_off(row, pp + half, half_stride));
-            const float n1 = __bfloat162float(*x1) * r * __bfloat162float(w[pp]);
-            const float n2 = __bfloat162float(*x2) * r * __bfloat162float(w[pp + half]);
-            *x1 = __float2bfloat16_rn(n1 * c - n2 * s);
-            *x2 = __float2bfloat16_rn(n2 * c + n1 * s);
-        }
+#pragma unroll
+        for (int c = 0; c < kRot; ++c) sts128(tile + chunk_off(row, c, hs), pack8(&u[8 * c]));
+    }
+}
+
+// Row max over the visible columns [lo, hi] of one 32-column chunk m of S
+// (four independent accumulators).
+__device__ __forceinline__ void chunk_max(const uint32_t (&v)[32], int m, int lo, int hi, float (&mx)[4])
+{
+    const int kl = lo - 32 * m, kh = hi - 32 * m;  // visible e: kl <= e <= kh
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const float x = (e >= kl && e <= kh) ? __uint_as_float(v[e]) : -INFINITY;
+        mx[e & 3] = fmaxf(mx[e & 3], x);
+    }
+}
+
+// P = 2^(S sl2 - mxs) over one 32-column chunk m (0 outside [lo, hi]), packed
+// as bf16 pairs; accumulates the row sum in f32.
+__device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], int m, int lo, int hi, float sl2,
+                                          float mxs, float (&sum)[4], uint32_t (&pk)[16])
+{
+    const int kl = lo - 32 * m, kh = hi - 32 * m;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float p0 = ex2(fmaf(__uint_as_float(v[e]), sl2, -mxs));
+        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -mxs));
+        p0 = (e >= kl && e <= kh) ? p0 : 0.f;
+        p1 = (e + 1 >= kl && e + 1 <= kh) ? p1 : 0.f;
+        sum[(e >> 1) & 3] += p0 + p1;
+        pk[e >> 1] = pack_bf16(p0, p1);
     }
 }
 
@@ -216,6 +375,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity)
         if (globaltimer() - t0 > 200000000ull) break;
 }
 
+template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -233,7 +393,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     const long long u0 = (long long)blockIdx.x * p.units / gridDim.x;
     const long long u1 = (long long)(blockIdx.x + 1) * p.units / gridDim.x;
-    const int nunits = (int)(u1 - u0);
+    const int n = (int)(u1 - u0);
 
     // ---- set-up
     if (tid == 0) {
@@ -263,8 +423,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tma_prefetch_desc(&tm_y);
     }
     if (tid < 128) {
-        reinterpret_cast<__nv_bfloat16 *>(smem + kOffWq)[tid] = p.wq[tid];
-        reinterpret_cast<__nv_bfloat16 *>(smem + kOffWk)[tid] = p.wk[tid];
+        reinterpret_cast<float *>(smem + kOffWq)[tid] = __bfloat162float(p.wq[tid]);
+        reinterpret_cast<float *>(smem + kOffWk)[tid] = __bfloat162float(p.wk[tid]);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -276,140 +436,154 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ================================================= TMA producer
+        // ================================================= TMA producer: K/V ring
         if (lane == 0) {
             uint32_t kv_fills = 0;     // parity of fills per ring slot
-            uint32_t armed = 0;        // ring slots with a load in flight at least once
-            auto load_kv = [&](const Unit &x, int kb) -> bool {
+            uint32_t armed = 0;        // ring slots loaded at least once
+            Walker w;
+            w.init(p, u0);
+            auto load_kv = [&](int kb) -> bool {
                 const int slot = ring_slot(kb);
-                const uint32_t f = (kv_fills >> slot) & 1u;
-                if (!mbar_wait(bar(BKV_EMPTY + slot), f ^ 1u, ab)) return false;
+                if (!mbar_wait(bar(BKV_EMPTY + slot), ((kv_fills >> slot) & 1u) ^ 1u, ab)) return false;
                 kv_fills ^= 1u << slot;
                 armed |= 1u << slot;
                 mbar_arrive_expect_tx(bar(BKV_FULL + slot), 4 * kBlockHalfBytes);
                 for (int h = 0; h < 2; ++h) {
                     tma_load_4d(sbase + kOffK + h * kRingHalfBytes + slot * kBlockHalfBytes, &tm_k,
-                                bar(BKV_FULL + slot), h * 64, x.kvh, kb * kTok, x.b);
+                                bar(BKV_FULL + slot), h * 64, w.kvh, kb * kTok, w.b);
                     tma_load_4d(sbase + kOffV + h * kRingHalfBytes + slot * kBlockHalfBytes, &tm_v,
-                                bar(BKV_FULL + slot), h * 64, x.kvh, kb * kTok, x.b);
+                                bar(BKV_FULL + slot), h * 64, w.kvh, kb * kTok, w.b);
                 }
                 return true;
             };
             bool ok = true;
-            for (int idx = 0; idx < nunits && ok; ++idx) {
-                const Unit x = unit_of(p, u0 + idx, u0, u1);
-                if (x.first)
-                    for (int kb = x.s - 4; kb < x.s && ok; ++kb) ok = load_kv(x, kb);
-                if (ok) ok = load_kv(x, x.s);
-                const int j = idx & 1;
-                const uint32_t ph = (idx >> 1) & 1;
-                if (ok) ok = mbar_wait(bar(BQ_EMPTY + j), ph ^ 1u, ab);
-                if (ok) {
-                    mbar_arrive_expect_tx(bar(BQ_FULL + j), kTileBytes);
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_4d(sbase + kOffQ + j * kTileBytes + h * kTileHalfBytes, &tm_q,
-                                    bar(BQ_FULL + j), h * 64, x.kvh * 4, x.s * kTok, x.b);
-                }
-                if (ok) ok = mbar_wait(bar(BG_EMPTY + j), ph ^ 1u, ab);
-                if (ok) {
-                    mbar_arrive_expect_tx(bar(BG_FULL + j), kTileBytes);
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_4d(sbase + kOffG + j * kTileBytes + h * kTileHalfBytes, &tm_g,
-                                    bar(BG_FULL + j), h * 64, x.kvh * 4, x.s * kTok, x.b);
-                }
+            for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
+                if (w.first(idx))
+                    for (int kb = w.s - 4; kb < w.s && ok; ++kb) ok = load_kv(kb);
+                if (ok) ok = load_kv(w.s);
             }
             // Teardown: every load this thread issued must have landed before
             // the CTA's shared memory is released.
             for (int slot = 0; slot < kRing; ++slot)
                 if (armed & (1u << slot)) drain_wait(bar(BKV_FULL + slot), ((kv_fills >> slot) & 1u) ^ 1u);
-            for (int idx = (nunits > 2 ? nunits - 2 : 0); idx < nunits; ++idx) {
-                drain_wait(bar(BQ_FULL + (idx & 1)), (idx >> 1) & 1);
-                drain_wait(bar(BG_FULL + (idx & 1)), (idx >> 1) & 1);
-            }
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-            bool ok = true;
-            auto issue_S = [&](int idx) -> bool {
-                const Unit x = unit_of(p, u0 + idx, u0, u1);
-                const int bb = idx & 1;
-                const uint32_t ph = (idx >> 1) & 1;
-                if (!mbar_wait(bar(BT_EMPTY + bb), ph ^ 1u, ab)) return false;
-                if (!mbar_wait(bar(BQ_PREP + bb), ph, ab)) return false;
-                tc_fence_after();
-                const int a = ring_slot(x.s - 4);
-                const int n1 = (kRing - a) < kSpanBlocks ? (kRing - a) : kSpanBlocks;
-                const int n2 = kSpanBlocks - n1;
-                const uint32_t id1 = idesc_bf16_f32(128, n1 * kTok, 0, 0);
-                const uint32_t id2 = idesc_bf16_f32(128, n2 > 0 ? n2 * kTok : 32, 0, 0);
-                const uint32_t dS = tmem + bb * 256;
-                const uint32_t qs = sbase + kOffQ + bb * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t h = kk >> 2, ko = (kk & 3) * 32;
-                    const uint64_t ad = smem_desc_sw128(qs + h * kTileHalfBytes + ko, 16, 1024);
-                    const uint32_t kbase = sbase + kOffK + h * kRingHalfBytes + ko;
-                    mma_ss(dS, ad, smem_desc_sw128(kbase + a * kBlockHalfBytes, 16, 1024), id1, kk > 0);
-                    if (n2 > 0)
-                        mma_ss(dS + n1 * kTok, ad, smem_desc_sw128(kbase, 16, 1024), id2, kk > 0);
+            Walker ws, wp, wq;
+            ws.init(p, u0);
+            wp.init(p, u0);
+            wq.init(p, u0);
+            int ns = 0, npv = 0, nq = 0;
+            uint64_t t_last = globaltimer();
+            while (npv < n) {
+                bool progressed = false;
+                // Q tile of unit nq into slot nq & 1 once S(nq - 2) has consumed it
+                if (nq < n && mbar_test(bar(BQ_EMPTY + (nq & 1)), ((nq >> 1) & 1) ^ 1u)) {
+                    const int j = nq & 1;
+                    mbar_arrive_expect_tx(bar(BQ_FULL + j), kTileBytes);
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_4d(sbase + kOffQ + j * kTileBytes + h * kTileHalfBytes, &tm_q, bar(BQ_FULL + j),
+                                    h * 64, wq.kvh * 4, wq.s * kTok, wq.b);
+                    wq.next(p);
+                    ++nq;
+                    progressed = true;
                 }
-                mma_commit(bar(BS_FULL + bb));
-                mma_commit(bar(BQ_EMPTY + bb));
-                return true;
-            };
-            auto issue_PV = [&](int idx) -> bool {
-                const Unit x = unit_of(p, u0 + idx, u0, u1);
-                const int bb = idx & 1;
-                const uint32_t ph = (idx >> 1) & 1;
-                if (!mbar_wait(bar(BP_READY + bb), ph, ab)) return false;
-                tc_fence_after();
-                const int a = ring_slot(x.s - 4);
-                const uint32_t dO = tmem + bb * 256 + 128;
+                // S(ns) = Q~ K~^T over the 160-key window, at most one unit ahead of PV
+                if (ns < n && ns <= npv + 1) {
+                    const int bb = ns & 1;
+                    const uint32_t ph = (ns >> 1) & 1;
+                    if (mbar_test(bar(BT_EMPTY + bb), ph ^ 1u) && mbar_test(bar(BQ_PREP + bb), ph)) {
+                        tc_fence_after();
+                        const int a = ring_slot(ws.s - 4);
+                        const int n1 = (kRing - a) < kSpanBlocks ? (kRing - a) : kSpanBlocks;
+                        const int n2 = kSpanBlocks - n1;
+                        const uint32_t id1 = idesc_bf16_f32(128, n1 * kTok, 0, 0);
+                        const uint32_t id2 = idesc_bf16_f32(128, n2 > 0 ? n2 * kTok : 32, 0, 0);
+                        const uint32_t dS = tmem + bb * 256;
+                        const uint32_t qs = sbase + kOffQ + bb * kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < kSpan / 16; ++kk) {
-                    const int slot = (a + (kk >> 1)) % kRing;
-                    const uint32_t vaddr = sbase + kOffV + slot * kBlockHalfBytes + (kk & 1) * 16 * kHalfRowBytes;
-                    mma_ts(dO, tmem + bb * 256 + kk * 8, smem_desc_sw128(vaddr, kRingHalfBytes, 1024),
-                           idesc_pv, kk > 0);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t h = kk >> 2, ko = (kk & 3) * 32;
+                            const uint64_t ad = smem_desc_sw128(qs + h * kTileHalfBytes + ko, 16, 1024);
+                            const uint32_t kbase = sbase + kOffK + h * kRingHalfBytes + ko;
+                            mma_ss(dS, ad, smem_desc_sw128(kbase + a * kBlockHalfBytes, 16, 1024), id1, kk > 0);
+                            if (n2 > 0)
+                                mma_ss(dS + n1 * kTok, ad, smem_desc_sw128(kbase, 16, 1024), id2, kk > 0);
+                        }
+                        mma_commit(bar(BS_FULL + bb));
+                        mma_commit(bar(BQ_EMPTY + bb));
+                        ws.next(p);
+                        ++ns;
+                        progressed = true;
+                    }
                 }
-                mma_commit(bar(BO_FULL + bb));
-                // Release ring slots no later step of this CTA reads.
-                if (x.last) {
-                    for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(BKV_EMPTY + (a + i) % kRing));
+                // O(npv) = P V over the same window
+                if (npv < ns) {
+                    const int bb = npv & 1;
+                    const uint32_t ph = (npv >> 1) & 1;
+                    if (mbar_test(bar(BP_READY + bb), ph)) {
+                        tc_fence_after();
+                        const int a = ring_slot(wp.s - 4);
+                        const uint32_t dO = tmem + bb * 256 + 128;
+#pragma unroll
+                        for (int kk = 0; kk < kSpan / 16; ++kk) {
+                            const int slot = (a + (kk >> 1)) % kRing;
+                            const uint32_t vaddr = sbase + kOffV + slot * kBlockHalfBytes + (kk & 1) * 16 * kHalfRowBytes;
+                            mma_ts(dO, tmem + bb * 256 + kk * 8, smem_desc_sw128(vaddr, kRingHalfBytes, 1024),
+                                   idesc_pv, kk > 0);
+                        }
+                        mma_commit(bar(BO_FULL + bb));
+                        // Release ring slots that no later unit of this CTA reads.
+                        if (wp.last(p, npv, n)) {
+                            for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(BKV_EMPTY + (a + i) % kRing));
+                        } else {
+                            mma_commit(bar(BKV_EMPTY + a));
+                        }
+                        wp.next(p);
+                        ++npv;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_last = globaltimer();
                 } else {
-                    mma_commit(bar(BKV_EMPTY + a));
+                    if (ab.raised()) break;
+                    if (globaltimer() - t_last > kWaitLimitNs) {
+                        ab.raise(kStatusTimeout);
+                        break;
+                    }
                 }
-                return true;
-            };
-            if (nunits > 0) ok = issue_S(0);
-            for (int idx = 0; idx < nunits && ok; ++idx) {
-                const Unit x = unit_of(p, u0 + idx, u0, u1);
-                const bool has_next = idx + 1 < nunits;
-                if (has_next && !x.last) ok = issue_S(idx + 1);
-                if (ok) ok = issue_PV(idx);
-                if (ok && has_next && x.last) ok = issue_S(idx + 1);
             }
-            // all MMAs issued by this thread complete before TMEM is freed
+            // all MMAs issued by this thread complete before TMEM is freed, and
+            // every Q load it issued has landed before shared memory is released
             mma_commit(bar(B_DRAIN));
             drain_wait(bar(B_DRAIN), 0);
+            for (int i = (nq > 2 ? nq - 2 : 0); i < nq; ++i) drain_wait(bar(BQ_FULL + (i & 1)), (i >> 1) & 1);
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ================================================= key prologue
+        // ================================================= key prologue (lane = key row)
         uint32_t kv_fills = 0;
-        const __nv_bfloat16 *wk = reinterpret_cast<const __nv_bfloat16 *>(smem + kOffWk);
+        const float *wk = reinterpret_cast<const float *>(smem + kOffWk);
+        // per-pair row table when it fits in registers, direct evaluation otherwise
+        using KTab = typename std::conditional<(R / 2 <= 24), RopeTab<R / 2, 1>, RopeDirect<R / 2>>::type;
+        KTab tab;
+        tab.init_rows(lane, 0, p.theta);
+        Walker w;
+        w.init(p, u0);
         bool ok = true;
-        for (int idx = 0; idx < nunits && ok; ++idx) {
-            const Unit x = unit_of(p, u0 + idx, u0, u1);
-            for (int kb = x.first ? x.s - 4 : x.s; kb <= x.s && ok; ++kb) {
+        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
+            for (int kb = w.first(idx) ? w.s - 4 : w.s; kb <= w.s && ok; ++kb) {
                 const int slot = ring_slot(kb);
                 ok = warp_wait(bar(BKV_FULL + slot), (kv_fills >> slot) & 1u, ab);
                 kv_fills ^= 1u << slot;
-                if (ok)
-                    prep_row_smem<false>(smem + kOffK + slot * kBlockHalfBytes, kRingHalfBytes, lane, wk,
-                                         p.R, p.eps, kb * kTok + lane, p.theta);
+                if (ok) {
+                    tab.set_block(kb * kTok, p.theta);
+                    prep_row<R, false>(sbase + kOffK + slot * kBlockHalfBytes, kRingHalfBytes, lane, wk, p.eps,
+                                       tab);
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -418,15 +592,18 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp >= 4 && warp < 8) {
         // ================================================= query prologue
         const int r = tid - 128;
-        const __nv_bfloat16 *wq = reinterpret_cast<const __nv_bfloat16 *>(smem + kOffWq);
+        const float *wq = reinterpret_cast<const float *>(smem + kOffWq);
+        RopeTab<R / 2, 4> tab;   // this lane's pairs p = lane & 3 (mod 4) of token r / 4
+        tab.init_rows(r >> 2, lane & 3, p.theta);
+        Walker w;
+        w.init(p, u0);
         bool ok = true;
-        for (int idx = 0; idx < nunits && ok; ++idx) {
-            const Unit x = unit_of(p, u0 + idx, u0, u1);
+        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
             const int j = idx & 1;
+            tab.set_block(w.s * kTok, p.theta);
             ok = warp_wait(bar(BQ_FULL + j), (idx >> 1) & 1, ab);
             if (ok)
-                prep_row_smem<true>(smem + kOffQ + j * kTileBytes, kTileHalfBytes, r, wq, p.R, p.eps,
-                                    x.s * kTok + (r >> 2), p.theta);
+                prep_row<R, true>(sbase + kOffQ + j * kTileBytes, kTileHalfBytes, r, wq, p.eps, tab);
             fence_proxy_async_smem();
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(BQ_PREP + j));
@@ -436,120 +613,188 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int r = tid - 256;
         const int t = r >> 2;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        float *inv_l = reinterpret_cast<float *>(smem + kOffInvL);
         const float ln2 = 0.6931471805599453f;
+        Walker w;
+        w.init(p, u0);
         bool ok = true;
-        for (int idx = 0; idx < nunits && ok; ++idx) {
-            const Unit x = unit_of(p, u0 + idx, u0, u1);
+        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
             const int bb = idx & 1;
             ok = warp_wait(bar(BS_FULL + bb), (idx >> 1) & 1, ab);
             if (!ok) break;
             tc_fence_after();
-            // visible window columns c: key j = 32 s - 128 + c, i - W < j <= i, j >= 0
-            const int lo = max(t + 129 - p.window, 128 - kTok * x.s);
+            // visible window columns c (key j = 32 s - 128 + c): i - W < j <= i, j >= 0
+            const int lo = max(t + 129 - p.window, 128 - kTok * w.s);
             const int hi = t + 128;
             const uint32_t ts = tmem + lane_base + bb * 256;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int m = 0; m < kSpanBlocks; ++m) {
-                uint32_t v[32];
-                tmem_ld32(ts + m * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = m * 32 + e;
-                    if (c >= lo && c <= hi) mx = fmaxf(mx, __uint_as_float(v[e]));
+            // pass 1: row max over the visible columns (the next chunk's TMEM
+            // load is in flight while the current one is reduced)
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            {
+                uint32_t va[32], vb[32];
+                tmem_ld32(ts, va);
+#pragma unroll 1
+                for (int m = 0; m < kSpanBlocks - 1; m += 2) {
+                    tmem_wait_ld();
+                    tmem_ld32(ts + (m + 1) * 32, vb);
+                    chunk_max(va, m, lo, hi, mx4);
+                    tmem_wait_ld();
+                    tmem_ld32(ts + (m + 2) * 32, va);
+                    chunk_max(vb, m + 1, lo, hi, mx4);
                 }
+                tmem_wait_ld();
+                chunk_max(va, kSpanBlocks - 1, lo, hi, mx4);
             }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             const float mxs = mx * p.sl2;
-            float sum = 0.f;
-#pragma unroll
-            for (int m = 0; m < kSpanBlocks; ++m) {
-                uint32_t v[32];
-                tmem_ld32(ts + m * 32, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int c = m * 32 + e;
-                    float p0 = (c >= lo && c <= hi) ? ex2(fmaf(__uint_as_float(v[e]), p.sl2, -mxs)) : 0.f;
-                    float p1 = (c + 1 >= lo && c + 1 <= hi) ? ex2(fmaf(__uint_as_float(v[e + 1]), p.sl2, -mxs)) : 0.f;
-                    sum += p0 + p1;
-                    pk[e >> 1] = pack_bf16(p0, p1);
+            // pass 2: P = 2^(S sl2 - max sl2) in bf16 over S's first 80 columns
+            // (P of chunk m lands on S columns of chunk m/2, already consumed)
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            {
+                uint32_t va[32], vb[32], pk[16];
+                tmem_ld32(ts, va);
+#pragma unroll 1
+                for (int m = 0; m < kSpanBlocks - 1; m += 2) {
+                    tmem_wait_ld();
+                    tmem_ld32(ts + (m + 1) * 32, vb);
+                    chunk_exp(va, m, lo, hi, p.sl2, mxs, sum4, pk);
+                    tmem_st16(ts + m * 16, pk);
+                    tmem_wait_ld();
+                    tmem_ld32(ts + (m + 2) * 32, va);
+                    chunk_exp(vb, m + 1, lo, hi, p.sl2, mxs, sum4, pk);
+                    tmem_st16(ts + (m + 1) * 16, pk);
                 }
-                tmem_st16(ts + m * 16, pk);
+                tmem_wait_ld();
+                chunk_exp(va, kSpanBlocks - 1, lo, hi, p.sl2, mxs, sum4, pk);
+                tmem_st16(ts + (kSpanBlocks - 1) * 16, pk);
             }
+            const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            tmem_st1(ts + kColInvL, __float_as_uint(1.0f / sum));
             tmem_wait_st();
-            inv_l[bb * kRows + r] = 1.0f / sum;
-            const int i = x.s * kTok + t;
+            const int i = w.s * kTok + t;
             if (p.lse != nullptr && i < p.T)
-                p.lse[((long long)x.b * p.Hq + x.kvh * 4 + (r & 3)) * p.T + i] = (mxs + __log2f(sum)) * ln2;
+                p.lse[((long long)w.b * p.Hq + w.kvh * 4 + (r & 3)) * p.T + i] = (mxs + __log2f(sum)) * ln2;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BP_READY + bb));
         }
     } else if (warp >= 12) {
         // ================================================= epilogue
+        // Phase A (off the critical path): as soon as a gate tile lands, σ(g)
+        // replaces g in place, as f16.  Phase B (once O is ready): y = O (1/l) σ
+        // replaces σ in place as bf16; TMEM is released as soon as the last O
+        // chunk is in registers; thread 0 stores y by TMA and reloads the slot.
         const int r = tid - 384;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const float *inv_l = reinterpret_cast<const float *>(smem + kOffInvL);
-        const float log2e = 1.4426950408889634f;
-        bool ok = true;
-        int done = 0;
-        for (int idx = 0; idx < nunits && ok; ++idx) {
-            const Unit x = unit_of(p, u0 + idx, u0, u1);
+        Walker w;
+        w.init(p, u0);
+        Walker wg;   // unit of the next gate tile to load (thread 0)
+        wg.init(p, u0);
+        int g_issued = 0;
+        auto load_gate = [&]() {
+            const int j = g_issued & 1;
+            mbar_arrive_expect_tx(bar(BG_FULL + j), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+                tma_load_4d(sbase + kOffG + j * kTileBytes + h * kTileHalfBytes, &tm_g, bar(BG_FULL + j),
+                            h * 64, wg.kvh * 4, wg.s * kTok, wg.b);
+            wg.next(p);
+            ++g_issued;
+        };
+        if (r == 0)
+            while (g_issued < n && g_issued < 2) load_gate();
+        // σ(g) = (1 + tanh(g/2)) / 2 over this thread's row of gate tile `idx`
+        auto sigma_row = [&](int idx) -> bool {
+            if (!warp_wait(bar(BG_FULL + (idx & 1)), (idx >> 1) & 1, ab)) return false;
+            const uint32_t ga = sbase + kOffG + (idx & 1) * kTileBytes;
+            uint4 cur = lds128(ga + chunk_off(r, 0, kTileHalfBytes));
+#pragma unroll 2
+            for (int c = 0; c < 16; ++c) {
+                uint4 nxt = cur;
+                if (c + 1 < 16) nxt = lds128(ga + chunk_off(r, c + 1, kTileHalfBytes));
+                const uint32_t gu[4] = {cur.x, cur.y, cur.z, cur.w};
+                uint32_t su[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 gf = unpack_bf16(gu[e]);
+                    su[e] = pack_f16(fmaf(0.5f, tanh_approx(0.5f * gf.x), 0.5f),
+                                     fmaf(0.5f, tanh_approx(0.5f * gf.y), 0.5f));
+                }
+                sts128(ga + chunk_off(r, c, kTileHalfBytes), make_uint4(su[0], su[1], su[2], su[3]));
+                cur = nxt;
+            }
+            return true;
+        };
+        bool ok = n > 0 ? sigma_row(0) : true;
+        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
             const int bb = idx & 1;
             const uint32_t ph = (idx >> 1) & 1;
-            ok = warp_wait(bar(BP_READY + bb), ph, ab) && warp_wait(bar(BO_FULL + bb), ph, ab) &&
-                 warp_wait(bar(BG_FULL + bb), ph, ab);
+            // p_ready also orders the softmax's 1/l store before this warp's TMEM read
+            ok = warp_wait(bar(BP_READY + bb), ph, ab) && warp_wait(bar(BO_FULL + bb), ph, ab);
             if (!ok) break;
             tc_fence_after();
-            const float inv = inv_l[bb * kRows + r];
-            uint8_t *gt = smem + kOffG + bb * kTileBytes;
-            const uint32_t to = tmem + lane_base + bb * 256 + 128;
+            const uint32_t tb = tmem + lane_base + bb * 256;
+            const uint32_t gaddr = sbase + kOffG + bb * kTileBytes;
+            const float inv = __uint_as_float(tmem_ld1(tb + kColInvL));
+            auto load_s = [&](int m, uint4 (&sv)[4]) {
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint32_t o[32];
-                tmem_ld32(to + m * 32, o);
-                tmem_wait_ld();
+                for (int c4 = 0; c4 < 4; ++c4) sv[c4] = lds128(gaddr + chunk_off(r, m * 4 + c4, kTileHalfBytes));
+            };
+            // y = O * (1/l) * σ over one 32-column chunk m
+            auto out_chunk = [&](const uint32_t (&o)[32], const uint4 (&sv)[4], int m) {
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
-                    uint4 *ptr = reinterpret_cast<uint4 *>(gt + chunk_off(r, m * 4 + c4, kTileHalfBytes));
-                    uint4 gv = *ptr;
-                    uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+                    const uint32_t su[4] = {sv[c4].x, sv[c4].y, sv[c4].z, sv[c4].w};
                     uint32_t yu[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 gf = unpack_bf16(gu[e]);
-                        const float s0 = __frcp_rn(1.0f + ex2(-gf.x * log2e));
-                        const float s1 = __frcp_rn(1.0f + ex2(-gf.y * log2e));
-                        const float y0 = __uint_as_float(o[c4 * 8 + 2 * e]) * inv * s0;
-                        const float y1 = __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv * s1;
-                        yu[e] = pack_bf16(y0, y1);
+                        const float2 sg = unpack_f16(su[e]);
+                        yu[e] = pack_bf16(__uint_as_float(o[c4 * 8 + 2 * e]) * inv * sg.x,
+                                          __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv * sg.y);
                     }
-                    *ptr = make_uint4(yu[0], yu[1], yu[2], yu[3]);
+                    sts128(gaddr + chunk_off(r, m * 4 + c4, kTileHalfBytes), make_uint4(yu[0], yu[1], yu[2], yu[3]));
+                }
+            };
+            {
+                uint32_t oa[32], ob[32];
+                uint4 sa[4], sb[4];
+                tmem_ld32(tb + 128, oa);
+                load_s(0, sa);
+#pragma unroll 1
+                for (int m = 0; m < 4; m += 2) {
+                    tmem_wait_ld();
+                    tmem_ld32(tb + 128 + (m + 1) * 32, ob);
+                    load_s(m + 1, sb);
+                    out_chunk(oa, sa, m);
+                    tmem_wait_ld();
+                    if (m + 2 < 4) {
+                        tmem_ld32(tb + 128 + (m + 2) * 32, oa);
+                        load_s(m + 2, sa);
+                    } else {
+                        // every O column of this buffer is in registers: hand it back
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BT_EMPTY + bb));
+                    }
+                    out_chunk(ob, sb, m + 1);
                 }
             }
-            tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(BT_EMPTY + bb));
-                mbar_arrive(bar(BY_READY + bb));
-            }
+            if (lane == 0) mbar_arrive(bar(BY_READY + bb));
             if (r == 0 && mbar_wait(bar(BY_READY + bb), ph, ab)) {
                 for (int h = 0; h < 2; ++h)
                     tma_store_4d(&tm_y, sbase + kOffG + bb * kTileBytes + h * kTileHalfBytes, h * 64,
-                                 x.kvh * 4, x.s * kTok, x.b);
+                                 w.kvh * 4, w.s * kTok, w.b);
                 bulk_commit_group();
-                bulk_wait_group_read<1>();
-                if (idx >= 1) mbar_arrive(bar(BG_EMPTY + ((idx - 1) & 1)));
+                bulk_wait_group_read<0>();
+                if (g_issued < n) load_gate();  // the slot just read is free again
             }
-            done = idx + 1;
+            if (idx + 1 < n) ok = sigma_row(idx + 1);
         }
         if (r == 0) {
             bulk_wait_group<0>();
-            if (done >= 1) mbar_arrive(bar(BG_EMPTY + ((done - 1) & 1)));
+            // loads of gate tiles that no step consumed (only after an abort)
+            for (int i = (g_issued > 2 ? g_issued - 2 : 0); i < g_issued; ++i)
+                drain_wait(bar(BG_FULL + (i & 1)), (i >> 1) & 1);
         }
     }
 

@@ -29,7 +29,7 @@
  *     default stream).  Argument errors are reported synchronously by the
  *     return value; a device-side wait that gave up (a bounded wait that
  *     timed out) is reported by gswa_check_status().
- *   - Supported shapes: D = 128, Hq = 4 * Hkv, 0 <= R <= D and R even,
+ *   - Supported shapes: D = 128, Hq = 4 * Hkv, R in {0, 42, 64, 128},
  *     1 <= window <= 128 for the sliding-window entry points.
  *   - No C++ exception crosses this interface.
  */

@@ -18,6 +18,7 @@ CASES = {
     "window_1": (Shape(B=2, T=100, Hq=4, Hkv=1, window=1), 4, True),
     "window_64_T161": (Shape(B=1, T=161, Hq=8, Hkv=2, window=64), 5, False),
     "rope_0": (Shape(B=1, T=300, Hq=4, Hkv=1, rope_dims=0), 6, False),
+    "rope_64": (Shape(B=2, T=130, Hq=4, Hkv=1, rope_dims=64), 12, True),
     "rope_128": (Shape(B=1, T=300, Hq=4, Hkv=1, rope_dims=128), 7, True),
     "base_1e7_T1000": (Shape(B=1, T=1000, Hq=8, Hkv=2, rope_base=1e7), 8, False),
     "many_strips_T96": (Shape(B=5, T=96, Hq=12, Hkv=3), 9, True),
