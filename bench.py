@@ -12,7 +12,8 @@ exchange step), so scaling is weak and `value` counts the tokens of all ranks.
 Timing: W untimed steps, then K steps between a barrier + cuda synchronize on
 both sides, CUDA events on the launching stream, max over ranks.  The inputs
 (> 600 MB for train_4k) are larger than the 126 MB L2, so every step streams
-them from HBM.  SM clocks are sampled with nvidia-smi during the timed region.
+them from HBM.  SM clocks and throttle reasons are sampled (NVML, read-only)
+during the timed region.
 """
 from __future__ import annotations
 
@@ -75,61 +76,85 @@ def swa_fwd_flops(s) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Reads NVML every ~2 ms from a thread (read-only queries; no setting is
+    touched); falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, device_index: int):
         self.dev = device_index
-        self.proc = None
-        self.lines = []
+        self.samples = []      # (sm_mhz, max_mhz, reasons)
+        self.stop = threading.Event()
+        self.thread = None
+        self.smi = None
+
+    def _handle(self, nv):
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _poll(self, nv, h):
+        masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), [n for n, m in masks if bits & m]))
+            except Exception:
+                break
+            time.sleep(0.002)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
             self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        except Exception:
+            try:
+                self.smi = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.dev}",
+                     "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                     "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                     "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.smi = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop.set()
+        if self.thread is not None:
             self.thread.join(timeout=5)
+        if self.smi is not None:
+            self.smi.terminate()
+            out, _ = self.smi.communicate(timeout=10)
+            names = [n for n, _ in self.REASONS]
+            for ln in out.splitlines():
+                parts = [x.strip() for x in ln.split(",")]
+                try:
+                    self.samples.append((float(parts[0]), float(parts[1]),
+                                         [n for n, v in zip(names, parts[2:6]) if v.lower() == "active"]))
+                except (ValueError, IndexError):
+                    continue
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [s[0] for s in self.samples]
+        reasons = sorted({r for s in self.samples for r in s[2]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.samples[-1][1],
+                "reasons": reasons, "samples": len(sm)}
 
 
 def make_step(ops, s, x, dev):
@@ -150,13 +175,15 @@ def make_step(ops, s, x, dev):
     return step, {"y": y, "lse": lse}, len(ops)
 
 
-def time_steps(step, K, W, stream, dist_on):
+def time_steps(step, K, W, stream, dist_on, sampler=None):
     for _ in range(W):
         step()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.__enter__()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -164,6 +191,8 @@ def time_steps(step, K, W, stream, dist_on):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.__exit__(None, None, None)
     if dist_on:
         torch.distributed.barrier()
     ms = e0.elapsed_time(e1)
@@ -260,7 +289,7 @@ def workload_config(s, name, ops, n):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="train_4k", choices=sorted(STEP_OPS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -289,8 +318,8 @@ def main():
     stream = torch.cuda.current_stream(dev)
     step, outs, launches_per_step = make_step(ops, s, x, dev)
 
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        ms = time_steps(step, args.steps, args.warmup, stream, dist_on)
+    clk = ClockSampler(torch.cuda.current_device())
+    ms = time_steps(step, args.steps, args.warmup, stream, dist_on, sampler=clk)
     clocks = clk.summary()
     if gca.gswa_check_status() != 0:
         raise RuntimeError("device status reports a timed-out wait")
