@@ -62,6 +62,7 @@ def lib():
             "full_attn_bwd": [S, P, P, P, P, P, P, P, P, P, P, P, P, P, U, P],
             "gswa_decode": [S, P, P, P, P, P, P, P, P, P, P, P, U, P],
             "full_decode": [S, P, P, P, P, P, P, P, P, P, U, P],
+            "gswa_qk_prep": [S, I, P, P, P, ctypes.c_int64, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -153,6 +154,18 @@ def full_attn_fwd(q, k, v, wq, wk, *, rope_dims=42, rope_base=1e4, eps=1e-6, sca
                                _ptr(y), _ptr(lse), _ptr(ws), nb, _stream(stream)),
            "full_attn_fwd")
     return y, lse
+
+
+def gswa_qk_prep(x, w, *, rope_dims=42, rope_base=1e4, eps=1e-6, pos0=0, out=None, stream=None):
+    """RMSNorm + partial RoPE of x [B, T, H, D] (bf16, cuda) at positions pos0 + t."""
+    torch = _dev(x, w, out)
+    B, T, H, D = x.shape
+    s = make_shape(B, T, H, H, D, 128, rope_dims, rope_base, eps)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().gswa_qk_prep(ctypes.byref(s), H, _ptr(x), _ptr(w), _ptr(out), pos0, _stream(stream)),
+           "gswa_qk_prep")
+    return out
 
 
 def _workspace(op, s, workspace, device):

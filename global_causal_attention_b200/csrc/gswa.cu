@@ -14,6 +14,8 @@
 #include "gswa.h"
 #include "ptx.cuh"
 #include "swa_fwd.cuh"
+#include "qk_prep.cuh"
+#include "full_fwd.cuh"
 
 namespace {
 
@@ -65,7 +67,11 @@ int device_setup(int *num_sms)
         } else if (set_smem(gswa::swa::swa_fwd_kernel<0>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::swa::swa_fwd_kernel<42>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::swa::swa_fwd_kernel<64>, gswa::swa::kSmemBytes) ||
-                   set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes)) {
+                   set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes) ||
+                   set_smem(gswa::full::full_fwd_kernel<0>, gswa::full::kSmemBytes) ||
+                   set_smem(gswa::full::full_fwd_kernel<42>, gswa::full::kSmemBytes) ||
+                   set_smem(gswa::full::full_fwd_kernel<64>, gswa::full::kSmemBytes) ||
+                   set_smem(gswa::full::full_fwd_kernel<128>, gswa::full::kSmemBytes)) {
             d.status = GSWA_ERR_LAUNCH;
         }
         if (d.status == GSWA_OK && g_encode == nullptr) {
@@ -117,6 +123,42 @@ void fill_theta(double *theta, int R, double base)
 {
     for (int p = 0; p < 64; ++p)
         theta[p] = (p < R / 2) ? std::pow(base, -2.0 * (double)p / (double)R) : 0.0;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Prepared-key workspace of the full causal forward: k~ [B, T, Hkv, D] bf16.
+size_t full_fwd_ws(const gswa_shape_t *s)
+{
+    return align256((size_t)s->B * s->T * s->Hkv * s->D * 2);
+}
+
+// RMSNorm + partial RoPE of x [B, T, H, 128] into out, positions pos0 + t.
+int launch_qk_prep(const gswa_shape_t *s, int H, const void *x, const void *w, void *out, long long pos0,
+                   cudaStream_t st, int num_sms)
+{
+    gswa::prep::Params pp;
+    std::memset(&pp, 0, sizeof pp);
+    pp.x = static_cast<const __nv_bfloat16 *>(x);
+    pp.out = static_cast<__nv_bfloat16 *>(out);
+    pp.w = static_cast<const __nv_bfloat16 *>(w);
+    pp.rows = (long long)s->B * s->T * H;
+    pp.T = s->T;
+    pp.H = H;
+    pp.pos0 = pos0;
+    pp.eps = s->eps;
+    fill_theta(pp.theta, s->rope_dims, s->rope_base);
+    const long long groups = (pp.rows + 31) / 32;
+    long long grid = (groups + gswa::prep::kWarps - 1) / gswa::prep::kWarps;
+    if (grid > 16LL * num_sms) grid = 16LL * num_sms;
+    const dim3 gr((unsigned)grid), bl(gswa::prep::kWarps * 32);
+    switch (s->rope_dims) {
+    case 0: gswa::prep::qk_prep_kernel<0><<<gr, bl, 0, st>>>(pp); break;
+    case 42: gswa::prep::qk_prep_kernel<42><<<gr, bl, 0, st>>>(pp); break;
+    case 64: gswa::prep::qk_prep_kernel<64><<<gr, bl, 0, st>>>(pp); break;
+    default: gswa::prep::qk_prep_kernel<128><<<gr, bl, 0, st>>>(pp); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
 }  // namespace
@@ -183,9 +225,73 @@ int full_attn_fwd(const gswa_shape_t *s, const void *q, const void *k, const voi
                   const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
                   size_t workspace_bytes, void *stream)
 {
-    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)y; (void)lse;
-    (void)workspace; (void)workspace_bytes; (void)stream;
-    return GSWA_ERR_UNIMPLEMENTED;
+    int rc = check_common(s);
+    if (rc != GSWA_OK) return rc;
+    if (!rope_dims_supported(s->rope_dims)) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)s->B * s->T == 0) return GSWA_OK;
+    if (!q || !k || !v || !w_q || !w_k || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return GSWA_ERR_MISALIGNED;
+    if (workspace == nullptr || workspace_bytes < full_fwd_ws(s)) return GSWA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // prepared keys once, into the workspace
+    rc = launch_qk_prep(s, s->Hkv, k, w_k, workspace, 0, st, num_sms);
+    if (rc != GSWA_OK) return rc;
+
+    CUtensorMap tq, tk, tv, ty;
+    if (encode_bthd(&tq, q, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&ty, y, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&tk, workspace, s->B, s->T, s->Hkv, s->D, 1, 128) ||
+        encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, 128))
+        return GSWA_ERR_INVALID_ARG;
+
+    gswa::full::Params p;
+    std::memset(&p, 0, sizeof p);
+    p.B = s->B;
+    p.T = s->T;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.nq = (s->T + gswa::full::kTok - 1) / gswa::full::kTok;
+    p.nkt = (s->T + gswa::full::kKeys - 1) / gswa::full::kKeys;
+    p.units = (long long)s->B * s->Hkv * p.nq;
+    p.eps = s->eps;
+    p.sl2 = s->scale * 1.4426950408889634f;
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.lse = lse;
+    fill_theta(p.theta, s->rope_dims, s->rope_base);
+
+    const long long grid = p.units < num_sms ? p.units : num_sms;
+    const dim3 gr((unsigned)grid), bl(gswa::full::kThreads);
+    const uint32_t sm = gswa::full::kSmemBytes;
+    switch (s->rope_dims) {
+    case 0: gswa::full::full_fwd_kernel<0><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
+    case 42: gswa::full::full_fwd_kernel<42><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
+    case 64: gswa::full::full_fwd_kernel<64><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
+    default: gswa::full::full_fwd_kernel<128><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
+int gswa_qk_prep(const gswa_shape_t *s, int H, const void *x, const void *w, void *out, int64_t pos0,
+                 void *stream)
+{
+    if (s == nullptr || H <= 0 || s->B < 0 || s->T < 0 || s->D != 128 || pos0 < 0)
+        return s && s->D != 128 ? GSWA_ERR_UNSUPPORTED_SHAPE : GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0)) return GSWA_ERR_INVALID_ARG;
+    if (!rope_dims_supported(s->rope_dims)) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)s->B * s->T == 0) return GSWA_OK;
+    if (!x || !w || !out) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    int rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    return launch_qk_prep(s, H, x, w, out, pos0, static_cast<cudaStream_t>(stream), num_sms);
 }
 
 int gswa_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
@@ -231,9 +337,11 @@ int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
 
 size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
 {
-    (void)op;
-    (void)s;
-    return 0;
+    if (s == nullptr || s->B < 0 || s->T < 0 || s->Hkv <= 0 || s->D <= 0) return 0;
+    switch (op) {
+    case GSWA_OP_FULL_FWD: return full_fwd_ws(s);
+    default: return 0;
+    }
 }
 
 int64_t gswa_kv_cache_bytes(int n_global_layers, int n_window_layers, int window, int Hkv, int D,

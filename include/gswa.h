@@ -92,7 +92,9 @@ int gswa_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void
 /*
  * Full causal attention forward of the 5 global layers (§2.1: global
  * layers attend over the whole context and drop the gate).  Same layouts
- * as gswa_fwd without g; shape->window is ignored.
+ * as gswa_fwd without g; shape->window is ignored.  Needs a workspace of
+ * gswa_workspace_bytes(GSWA_OP_FULL_FWD) bytes (device, 16-byte aligned):
+ * it receives the prepared keys.
  */
 int full_attn_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                   const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
@@ -139,6 +141,16 @@ int full_decode(const gswa_shape_t *shape, const void *q, const void *k, const v
                 const void *w_q, const void *w_k, void *k_cache, void *v_cache,
                 const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
                 void *stream);
+
+/*
+ * QK-RMSNorm + partial RoPE of a head tensor on its own (§2.1 Figure 3: the
+ * prologue of the attention core): out[b,t,h,:] = RoPE_{pos0+t}(RMSNorm(
+ * x[b,t,h,:]) * w).  x, out [B,T,H,D] bf16 (device; may not alias), w [D]
+ * bf16 (device).  Uses shape->B, T, D, rope_dims, rope_base, eps.  Fills
+ * decode caches, which hold prepared keys.
+ */
+int gswa_qk_prep(const gswa_shape_t *shape, int H, const void *x, const void *w, void *out,
+                 int64_t pos0, void *stream);
 
 /* Workspace bytes an operation needs for `shape` (0 when none). */
 size_t gswa_workspace_bytes(int op, const gswa_shape_t *shape);
