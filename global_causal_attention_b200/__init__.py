@@ -55,19 +55,21 @@ def lib():
             raise ImportError(f"{LIB_PATH} is missing: run global_causal_attention_b200/build.py")
         L = ctypes.CDLL(LIB_PATH)
         P, S, I, U = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.c_int, ctypes.c_size_t
+        # (shape, then the pointer arguments, then workspace bytes and the stream)
         sig = {
-            "gswa_fwd": [S, P, P, P, P, P, P, P, P, P, U, P],
-            "full_attn_fwd": [S, P, P, P, P, P, P, P, P, U, P],
-            "gswa_bwd": [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, U, P],
-            "full_attn_bwd": [S, P, P, P, P, P, P, P, P, P, P, P, P, P, U, P],
-            "gswa_decode": [S, P, P, P, P, P, P, P, P, P, P, P, U, P],
-            "full_decode": [S, P, P, P, P, P, P, P, P, P, U, P],
+            "gswa_fwd": [S] + [P] * 9 + [U, P],
+            "full_attn_fwd": [S] + [P] * 8 + [U, P],
+            "gswa_bwd": [S] + [P] * 16 + [U, P],
+            "full_attn_bwd": [S] + [P] * 14 + [U, P],
+            "gswa_decode": [S] + [P] * 11 + [U, P],
+            "full_decode": [S] + [P] * 10 + [U, P],
             "gswa_qk_prep": [S, I, P, P, P, ctypes.c_int64, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = I
+        L._gswa_signatures = sig
         L.gswa_workspace_bytes.argtypes = [I, S]
         L.gswa_workspace_bytes.restype = U
         L.gswa_kv_cache_bytes.argtypes = [I, I, I, I, I, I, ctypes.c_int64]
@@ -166,6 +168,37 @@ def gswa_qk_prep(x, w, *, rope_dims=42, rope_base=1e4, eps=1e-6, pos0=0, out=Non
     _check(lib().gswa_qk_prep(ctypes.byref(s), H, _ptr(x), _ptr(w), _ptr(out), pos0, _stream(stream)),
            "gswa_qk_prep")
     return out
+
+
+def gswa_decode(q, k, v, g, wq, wk, k_ring, v_ring, pos, *, rope_dims=42, rope_base=1e4, eps=1e-6,
+                scale=None, y=None, stream=None):
+    """One gated-SWA decode step over a ring cache [B, Hkv, W, D] (updated in place).
+    q, g [B, Hq, D], k, v [B, Hkv, D] bf16; pos [B] int64; returns y [B, Hq, D]."""
+    torch = _dev(q, k, v, g, wq, wk, k_ring, v_ring, pos, y)
+    B, Hq, D = q.shape
+    s = make_shape(B, 1, Hq, k.shape[1], D, k_ring.shape[2], rope_dims, rope_base, eps, scale)
+    if y is None:
+        y = torch.empty_like(q)
+    _check(lib().gswa_decode(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
+                             _ptr(k_ring), _ptr(v_ring), _ptr(pos), _ptr(y), None, 0, _stream(stream)),
+           "gswa_decode")
+    return y
+
+
+def full_decode(q, k, v, wq, wk, k_cache, v_cache, pos, *, rope_dims=42, rope_base=1e4, eps=1e-6,
+                scale=None, y=None, workspace=None, stream=None):
+    """One global-layer decode step over a linear cache [B, Hkv, Tmax, D] (row pos written)."""
+    torch = _dev(q, k, v, wq, wk, k_cache, v_cache, pos, y)
+    B, Hq, D = q.shape
+    s = make_shape(B, 1, Hq, k.shape[1], D, 128, rope_dims, rope_base, eps, scale,
+                   cache_len=k_cache.shape[2])
+    if y is None:
+        y = torch.empty_like(q)
+    ws, nb = _workspace(OP_FULL_DECODE, s, workspace, q.device)
+    _check(lib().full_decode(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk),
+                             _ptr(k_cache), _ptr(v_cache), _ptr(pos), _ptr(y), _ptr(ws), nb,
+                             _stream(stream)), "full_decode")
+    return y
 
 
 def _workspace(op, s, workspace, device):

@@ -1,0 +1,368 @@
+// decode.cuh -- one decode step of the ZGCM-1 attention core (§2.3: the SWA
+// layers keep a fixed 128-token window in the KV cache, the global layers
+// the whole sequence; autoregressive decoding is bound by memory bandwidth).
+//
+// Both paths prepare the new token's q and k (RMSNorm + partial RoPE at its
+// position), write the prepared k and the raw v into the cache, then attend.
+//
+//   gswa_decode: ring cache [B, Hkv, W, D]; position t lives in slot t mod W.
+//     One CTA per (sequence, KV head), one warp per query head of the group.
+//   full_decode: linear cache [B, Hkv, Tmax, D], split over the cache length:
+//     a prologue prepares q~ (f32, into the workspace) and appends k~, v; a
+//     chunk kernel computes, per 4096-key chunk, the partial (max, sum, O) of
+//     the 4 query heads (lanes = keys for q.k with q~ broadcast from shared
+//     memory, lanes = dims for P V with 8-byte coalesced value loads); a
+//     combine kernel merges the chunks by their log-sum-exp weights.
+#pragma once
+
+#include "ptx.cuh"
+#include "swa_fwd.cuh"
+
+namespace gswa {
+namespace dec {
+
+constexpr int kD = 128;
+constexpr int kChunk = 4096;          // keys per chunk of the full-cache split
+constexpr int kChunkWarps = 8;
+constexpr int kPartial = 4 + kD;      // m, l, (2 pad), o[128] per (chunk, head): o 16-byte aligned
+
+struct Params {
+    int B, Hq, Hkv, R;
+    int W;               // ring slots (sliding-window decode)
+    long long Tmax;      // linear cache length (full decode)
+    int nchunks;         // ceil(Tmax / kChunk)
+    float eps, sl2;      // softmax scale * log2(e)
+    const __nv_bfloat16 *q, *k, *v, *g, *wq, *wk;
+    __nv_bfloat16 *kc, *vc;   // caches (written at the new position)
+    const int64_t *pos;
+    __nv_bfloat16 *y;
+    float *qt;           // full decode: prepared queries [B, Hq, D] f32
+    float *part;         // full decode: partials [B, Hkv, nchunks, 4, kPartial]
+    double theta[64];
+};
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float warp_max(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+// RMSNorm then partial RoPE of one head row by one warp; lane l returns dims
+// 4l .. 4l+3 (f32).  `ubuf` is 128 floats of shared memory for the rotation.
+__device__ __forceinline__ float4 prep_head_warp(const __nv_bfloat16 *x, const __nv_bfloat16 *w, int R,
+                                                 float eps, long long pos, const double *theta,
+                                                 float *ubuf)
+{
+    const int lane = threadIdx.x & 31;
+    const uint2 raw = *reinterpret_cast<const uint2 *>(x + 4 * lane);
+    const uint2 wr = *reinterpret_cast<const uint2 *>(w + 4 * lane);
+    const float2 a = unpack_bf16(raw.x), b = unpack_bf16(raw.y);
+    const float2 wa = unpack_bf16(wr.x), wb = unpack_bf16(wr.y);
+    const float ss = warp_sum(a.x * a.x + a.y * a.y + b.x * b.x + b.y * b.y);
+    const float r = rsqrtf(ss * (1.0f / kD) + eps);
+    float u[4] = {a.x * r * wa.x, a.y * r * wa.y, b.x * r * wb.x, b.y * r * wb.y};
+    const int H = R / 2;
+    if (R > 0) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ubuf[4 * lane + e] = u[e];
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int d = 4 * lane + e;
+            if (d < R) {
+                const int pp = d < H ? d : d - H;
+                float c, s;
+                swa::rope_cs(theta[pp], (int)pos, c, s);
+                u[e] = d < H ? ubuf[d] * c - ubuf[d + H] * s : ubuf[d] * c + ubuf[d - H] * s;
+            }
+        }
+        __syncwarp();
+    }
+    return make_float4(u[0], u[1], u[2], u[3]);
+}
+
+// ----------------------------------------------------------------- sliding window
+__global__ void __launch_bounds__(128)
+swa_decode_kernel(const __grid_constant__ Params p)
+{
+    __shared__ __align__(16) float qt[4][kD];
+    __shared__ __align__(16) float ubuf[4][kD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv;
+    const int head = kvh * 4 + warp;
+    const long long pos = p.pos[b];
+    if (pos < 0) {
+        if (threadIdx.x == 0) atomicExch(&g_status, kStatusBadArg);
+        return;
+    }
+    const int W = p.W;
+    const int slot_new = (int)(pos % W);
+    const long long cbase = ((long long)b * p.Hkv + kvh) * W;   // first row of this (b, kvh) ring
+
+    const float4 q4 = prep_head_warp(p.q + ((long long)b * p.Hq + head) * kD, p.wq, p.R, p.eps, pos,
+                                     p.theta, ubuf[warp]);
+    *reinterpret_cast<float4 *>(&qt[warp][4 * lane]) = q4;
+    if (warp == 0) {
+        // the new key, prepared and rounded as the cache stores it
+        const float4 k4 = prep_head_warp(p.k + ((long long)b * p.Hkv + kvh) * kD, p.wk, p.R, p.eps, pos,
+                                         p.theta, ubuf[0]);
+        *reinterpret_cast<uint2 *>(p.kc + (cbase + slot_new) * kD + 4 * lane) =
+            make_uint2(pack_bf16(k4.x, k4.y), pack_bf16(k4.z, k4.w));
+    } else if (warp == 1) {
+        *reinterpret_cast<uint2 *>(p.vc + (cbase + slot_new) * kD + 4 * lane) =
+            *reinterpret_cast<const uint2 *>(p.v + ((long long)b * p.Hkv + kvh) * kD + 4 * lane);
+    }
+    __syncthreads();
+
+    // scores: lane owns slots lane + 32 i; slot s holds position pos - ((slot_new - s) mod W)
+    float sc[4];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int s = lane + 32 * i;
+        sc[i] = -INFINITY;
+        if (s < W) {
+            const int age = (slot_new - s + W) % W;
+            if (age <= pos) {
+                const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + (cbase + s) * kD);
+                float acc = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 kv = kr[c];
+                    const float4 qa = *reinterpret_cast<const float4 *>(&qt[warp][8 * c]);
+                    const float4 qb = *reinterpret_cast<const float4 *>(&qt[warp][8 * c + 4]);
+                    const float2 k0 = unpack_bf16(kv.x), k1 = unpack_bf16(kv.y), k2 = unpack_bf16(kv.z),
+                                 k3 = unpack_bf16(kv.w);
+                    acc = fmaf(qa.x, k0.x, fmaf(qa.y, k0.y, fmaf(qa.z, k1.x, fmaf(qa.w, k1.y, acc))));
+                    acc = fmaf(qb.x, k2.x, fmaf(qb.y, k2.y, fmaf(qb.z, k3.x, fmaf(qb.w, k3.y, acc))));
+                }
+                sc[i] = acc * p.sl2;
+            }
+        }
+        mx = fmaxf(mx, sc[i]);
+    }
+    mx = warp_max(mx);
+    float pr[4], l = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        pr[i] = sc[i] == -INFINITY ? 0.f : ex2(sc[i] - mx);
+        l += pr[i];
+    }
+    l = warp_sum(l);
+    // P V: lane owns dims 4 lane .. 4 lane + 3
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const int s = 32 * i + j;
+            const float ps = __shfl_sync(0xffffffffu, pr[i], j);
+            if (s < W && ps != 0.f) {
+                const uint2 vv = *reinterpret_cast<const uint2 *>(p.vc + (cbase + s) * kD + 4 * lane);
+                const float2 v0 = unpack_bf16(vv.x), v1 = unpack_bf16(vv.y);
+                o[0] = fmaf(ps, v0.x, o[0]);
+                o[1] = fmaf(ps, v0.y, o[1]);
+                o[2] = fmaf(ps, v1.x, o[2]);
+                o[3] = fmaf(ps, v1.y, o[3]);
+            }
+        }
+    }
+    const float inv = 1.0f / l;
+    const uint2 gr = *reinterpret_cast<const uint2 *>(p.g + ((long long)b * p.Hq + head) * kD + 4 * lane);
+    const float2 g0 = unpack_bf16(gr.x), g1 = unpack_bf16(gr.y);
+    auto sig = [](float x) { return 1.0f / (1.0f + ex2(-1.4426950408889634f * x)); };
+    *reinterpret_cast<uint2 *>(p.y + ((long long)b * p.Hq + head) * kD + 4 * lane) =
+        make_uint2(pack_bf16(o[0] * inv * sig(g0.x), o[1] * inv * sig(g0.y)),
+                   pack_bf16(o[2] * inv * sig(g1.x), o[3] * inv * sig(g1.y)));
+}
+
+// ----------------------------------------------------------------- full cache
+// Prologue: q~ of the 4 heads (f32, workspace) and k~, v appended at `pos`.
+__global__ void __launch_bounds__(128)
+full_decode_prep_kernel(const __grid_constant__ Params p)
+{
+    __shared__ __align__(16) float ubuf[4][kD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv;
+    const int head = kvh * 4 + warp;
+    const long long pos = p.pos[b];
+    if (pos < 0 || pos >= p.Tmax) {
+        if (threadIdx.x == 0) atomicExch(&g_status, kStatusBadArg);
+        return;
+    }
+    const float4 q4 = prep_head_warp(p.q + ((long long)b * p.Hq + head) * kD, p.wq, p.R, p.eps, pos,
+                                     p.theta, ubuf[warp]);
+    *reinterpret_cast<float4 *>(p.qt + ((long long)b * p.Hq + head) * kD + 4 * lane) = q4;
+    const long long row = ((long long)b * p.Hkv + kvh) * p.Tmax + pos;
+    if (warp == 0) {
+        const float4 k4 = prep_head_warp(p.k + ((long long)b * p.Hkv + kvh) * kD, p.wk, p.R, p.eps, pos,
+                                         p.theta, ubuf[0]);
+        *reinterpret_cast<uint2 *>(p.kc + row * kD + 4 * lane) =
+            make_uint2(pack_bf16(k4.x, k4.y), pack_bf16(k4.z, k4.w));
+    } else if (warp == 1) {
+        *reinterpret_cast<uint2 *>(p.vc + row * kD + 4 * lane) =
+            *reinterpret_cast<const uint2 *>(p.v + ((long long)b * p.Hkv + kvh) * kD + 4 * lane);
+    }
+}
+
+__device__ __forceinline__ uint64_t f2_bits(float a, float b)
+{
+    return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+
+// acc(2) += x(2) * s(broadcast)
+__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t x, float s)
+{
+    const uint64_t ss = f2_bits(s, s);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(ss));
+}
+
+// Chunk c of (b, kvh): partial softmax state of the 4 heads over keys
+// [c * kChunk, (c + 1) * kChunk) intersected with [0, pos].
+__global__ void __launch_bounds__(kChunkWarps * 32)
+full_decode_chunk_kernel(const __grid_constant__ Params p)
+{
+    __shared__ __align__(16) float qt[4][kD];
+    __shared__ float wm[kChunkWarps][4], wl[kChunkWarps][4];
+    __shared__ __align__(16) float wo[kChunkWarps][4][kD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
+    const long long pos = p.pos[b];
+    if (pos < 0 || pos >= p.Tmax || (long long)c * kChunk > pos) return;   // nothing to attend here
+    for (int i = threadIdx.x; i < 4 * kD; i += blockDim.x)
+        qt[i / kD][i % kD] = p.qt[((long long)b * p.Hq + kvh * 4) * kD + i];
+    __syncthreads();
+    const long long rowbase = ((long long)b * p.Hkv + kvh) * p.Tmax;
+    const long long k0 = (long long)c * kChunk;
+    const long long k1 = min(k0 + kChunk, pos + 1);   // exclusive end
+    const int per_warp = kChunk / kChunkWarps;
+    const long long w0 = k0 + (long long)warp * per_warp;
+    const long long w1 = min(w0 + per_warp, k1);
+
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running max (log2 units)
+    float l[4] = {0.f, 0.f, 0.f, 0.f};                          // this lane's keys' sums
+    uint64_t o[4][2];                                           // dims 4 lane..+3, as 2 pairs
+#pragma unroll
+    for (int h = 0; h < 4; ++h) o[h][0] = o[h][1] = 0;
+    for (long long t0 = w0; t0 < w1; t0 += 32) {
+        const long long key = t0 + lane;
+        float s[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (key < w1) {
+            const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + (rowbase + key) * kD);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int ch = 0; ch < 16; ++ch) {
+                const uint4 kv = kr[ch];
+                const float2 ka = unpack_bf16(kv.x), kb = unpack_bf16(kv.y), kc2 = unpack_bf16(kv.z),
+                             kd = unpack_bf16(kv.w);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float4 qa = *reinterpret_cast<const float4 *>(&qt[h][8 * ch]);
+                    const float4 qb = *reinterpret_cast<const float4 *>(&qt[h][8 * ch + 4]);
+                    float a = acc[h];
+                    a = fmaf(qa.x, ka.x, fmaf(qa.y, ka.y, fmaf(qa.z, kb.x, fmaf(qa.w, kb.y, a))));
+                    a = fmaf(qb.x, kc2.x, fmaf(qb.y, kc2.y, fmaf(qb.z, kd.x, fmaf(qb.w, kd.y, a))));
+                    acc[h] = a;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) s[h] = acc[h] * p.sl2;
+        }
+        float pr[4], alpha[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float tm = warp_max(s[h]);
+            const float mn = fmaxf(m[h], tm);
+            alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+            m[h] = mn;
+            pr[h] = (s[h] == -INFINITY) ? 0.f : ex2(s[h] - mn);
+            l[h] = l[h] * alpha[h] + pr[h];
+            const uint64_t a2 = f2_bits(alpha[h], alpha[h]);
+            asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][0]) : "l"(a2));
+            asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][1]) : "l"(a2));
+        }
+        const int nk = (int)min((long long)32, w1 - t0);
+        for (int j = 0; j < nk; ++j) {
+            const uint2 vv = *reinterpret_cast<const uint2 *>(p.vc + (rowbase + t0 + j) * kD + 4 * lane);
+            const float2 va = unpack_bf16(vv.x), vb = unpack_bf16(vv.y);
+            const uint64_t v01 = f2_bits(va.x, va.y), v23 = f2_bits(vb.x, vb.y);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float ps = __shfl_sync(0xffffffffu, pr[h], j);
+                ffma2(o[h][0], v01, ps);
+                ffma2(o[h][1], v23, ps);
+            }
+        }
+    }
+    // combine the warps of this chunk
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float lsum = warp_sum(l[h]);
+        if (lane == 0) {
+            wm[warp][h] = m[h];
+            wl[warp][h] = lsum;
+        }
+        float2 a = *reinterpret_cast<float2 *>(&o[h][0]), bq = *reinterpret_cast<float2 *>(&o[h][1]);
+        *reinterpret_cast<float4 *>(&wo[warp][h][4 * lane]) = make_float4(a.x, a.y, bq.x, bq.y);
+    }
+    __syncthreads();
+    // thread t: head t / 32... one warp per head: lanes cover dims 4 lane .. +3
+    if (warp < 4) {
+        const int h = warp;
+        float M = -INFINITY;
+        for (int w = 0; w < kChunkWarps; ++w) M = fmaxf(M, wm[w][h]);
+        float L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < kChunkWarps; ++w) {
+            if (wm[w][h] == -INFINITY) continue;
+            const float f = ex2(wm[w][h] - M);
+            L += wl[w][h] * f;
+            const float4 ow = *reinterpret_cast<const float4 *>(&wo[w][h][4 * lane]);
+            acc.x += ow.x * f;
+            acc.y += ow.y * f;
+            acc.z += ow.z * f;
+            acc.w += ow.w * f;
+        }
+        float *dst = p.part + ((((long long)b * p.Hkv + kvh) * p.nchunks + c) * 4 + h) * kPartial;
+        if (lane == 0) {
+            dst[0] = M;
+            dst[1] = L;
+        }
+        *reinterpret_cast<float4 *>(dst + 4 + 4 * lane) = acc;
+    }
+}
+
+// Merge the chunks of (b, head): y = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+__global__ void __launch_bounds__(kD)
+full_decode_combine_kernel(const __grid_constant__ Params p)
+{
+    const int b = blockIdx.x / p.Hq, head = blockIdx.x % p.Hq;
+    const int kvh = head / 4, h = head % 4;
+    const int d = threadIdx.x;
+    const long long pos = p.pos[b];
+    if (pos < 0 || pos >= p.Tmax) return;
+    const int nc = (int)(pos / kChunk) + 1;
+    const float *base = p.part + (((long long)b * p.Hkv + kvh) * p.nchunks * 4 + h) * kPartial;
+    float M = -INFINITY;
+    for (int c = 0; c < nc; ++c) M = fmaxf(M, base[(long long)c * 4 * kPartial]);
+    float L = 0.f, acc = 0.f;
+    for (int c = 0; c < nc; ++c) {
+        const float *pc = base + (long long)c * 4 * kPartial;
+        if (pc[0] == -INFINITY) continue;
+        const float f = ex2(pc[0] - M);
+        L += pc[1] * f;
+        acc += pc[4 + d] * f;
+    }
+    p.y[((long long)b * p.Hq + head) * kD + d] = __float2bfloat16_rn(acc / L);
+}
+
+}  // namespace dec
+}  // namespace gswa

@@ -16,6 +16,7 @@
 #include "swa_fwd.cuh"
 #include "qk_prep.cuh"
 #include "full_fwd.cuh"
+#include "decode.cuh"
 
 namespace {
 
@@ -126,6 +127,30 @@ void fill_theta(double *theta, int R, double base)
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of the full-cache decode: q~ [B, Hq, D] f32, then the chunk
+// partials [B, Hkv, nchunks, 4, kPartial] f32.
+size_t full_decode_ws(const gswa_shape_t *s)
+{
+    const size_t nch = ((size_t)s->cache_len + gswa::dec::kChunk - 1) / gswa::dec::kChunk;
+    return align256((size_t)s->B * s->Hq * s->D * 4) +
+           align256((size_t)s->B * s->Hkv * nch * 4 * gswa::dec::kPartial * 4);
+}
+
+void fill_dec(gswa::dec::Params &p, const gswa_shape_t *s)
+{
+    std::memset(&p, 0, sizeof p);
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.R = s->rope_dims;
+    p.W = s->window;
+    p.Tmax = s->cache_len;
+    p.nchunks = (int)((s->cache_len + gswa::dec::kChunk - 1) / gswa::dec::kChunk);
+    p.eps = s->eps;
+    p.sl2 = s->scale * 1.4426950408889634f;
+    fill_theta(p.theta, s->rope_dims, s->rope_base);
+}
 
 // Prepared-key workspace of the full causal forward: k~ [B, T, Hkv, D] bf16.
 size_t full_fwd_ws(const gswa_shape_t *s)
@@ -320,9 +345,35 @@ int gswa_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
                 const void *w_q, const void *w_k, void *k_ring, void *v_ring, const int64_t *pos,
                 void *y, void *workspace, size_t workspace_bytes, void *stream)
 {
-    (void)s; (void)q; (void)k; (void)v; (void)g; (void)w_q; (void)w_k; (void)k_ring;
-    (void)v_ring; (void)pos; (void)y; (void)workspace; (void)workspace_bytes; (void)stream;
-    return GSWA_ERR_UNIMPLEMENTED;
+    (void)workspace;
+    (void)workspace_bytes;
+    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0) return GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
+    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->window < 1 || s->window > 128 ||
+        s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
+        return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->B == 0) return GSWA_OK;
+    if (!q || !k || !v || !g || !w_q || !w_k || !k_ring || !v_ring || !pos || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(k_ring) ||
+        !aligned16(v_ring) || !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+        return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    int rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    gswa::dec::Params p;
+    fill_dec(p, s);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.g = static_cast<const __nv_bfloat16 *>(g);
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.kc = static_cast<__nv_bfloat16 *>(k_ring);
+    p.vc = static_cast<__nv_bfloat16 *>(v_ring);
+    p.pos = pos;
+    p.y = static_cast<__nv_bfloat16 *>(y);
+    gswa::dec::swa_decode_kernel<<<s->B * s->Hkv, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
 int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v,
@@ -330,9 +381,39 @@ int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
                 const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
                 void *stream)
 {
-    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)k_cache; (void)v_cache;
-    (void)pos; (void)y; (void)workspace; (void)workspace_bytes; (void)stream;
-    return GSWA_ERR_UNIMPLEMENTED;
+    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->cache_len < 1) return GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
+    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
+        return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->B == 0) return GSWA_OK;
+    if (!q || !k || !v || !w_q || !w_k || !k_cache || !v_cache || !pos || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+        return GSWA_ERR_MISALIGNED;
+    if (workspace == nullptr || workspace_bytes < full_decode_ws(s)) return GSWA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    int rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    gswa::dec::Params p;
+    fill_dec(p, s);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    p.pos = pos;
+    p.y = static_cast<__nv_bfloat16 *>(y);
+    p.qt = static_cast<float *>(workspace);
+    p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                       align256((size_t)s->B * s->Hq * s->D * 4));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
+    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkWarps * 32, 0, st>>>(p);
+    gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
 size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
@@ -340,6 +421,7 @@ size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
     if (s == nullptr || s->B < 0 || s->T < 0 || s->Hkv <= 0 || s->D <= 0) return 0;
     switch (op) {
     case GSWA_OP_FULL_FWD: return full_fwd_ws(s);
+    case GSWA_OP_FULL_DECODE: return s->cache_len > 0 ? full_decode_ws(s) : 0;
     default: return 0;
     }
 }
@@ -363,7 +445,7 @@ int gswa_check_status(void *stream)
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(gswa::g_status, &zero, sizeof zero) != cudaSuccess) return GSWA_ERR_LAUNCH;
-        return GSWA_ERR_TIMEOUT;
+        return v == gswa::kStatusBadArg ? GSWA_ERR_INVALID_ARG : GSWA_ERR_TIMEOUT;
     }
     return GSWA_OK;
 }

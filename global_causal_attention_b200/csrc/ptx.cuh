@@ -15,6 +15,7 @@ namespace gswa {
 __device__ int g_status;
 
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadArg = 2;   // a device-side argument (a decode position) was out of range
 // A wait gives up after this much wall time (the kernels' longest legitimate
 // wait is a few microseconds; profilers that serialise passes stay far below).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;

@@ -125,7 +125,9 @@ int full_attn_bwd(const gswa_shape_t *shape, const void *q, const void *k, const
  *     v_ring raw values.  The new token is written to slot pos mod W and is
  *     part of its own window; slots holding positions < 0 are ignored.
  *   pos [B] int64 (device): position of the new token of each sequence.
- *   y [B,Hq,D] bf16 (device, written).  shape->window = W = ring slots.
+ *   y [B,Hq,D] bf16 (device, written).  shape->window = W = ring slots
+ *   (1..128).  No workspace.  A negative pos skips that sequence and is
+ *   reported by gswa_check_status().
  */
 int gswa_decode(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                 const void *g, const void *w_q, const void *w_k, void *k_ring, void *v_ring,
@@ -134,8 +136,13 @@ int gswa_decode(const gswa_shape_t *shape, const void *q, const void *k, const v
 
 /*
  * One decode step of a global layer over a linear cache [B,Hkv,Tmax,D]
- * (Tmax = shape->cache_len): writes the new key/value at row pos and attends
- * over rows 0..pos.  Split over the cache length; needs a workspace.
+ * (Tmax = shape->cache_len): writes the prepared key and the value of the
+ * new token at row pos and attends over rows 0..pos (positions must lie in
+ * [0, Tmax); others skip the sequence and are reported by
+ * gswa_check_status()).  q, k, v, pos, y as in gswa_decode (no gate).
+ * Split over the cache length in 4096-key chunks whose partial softmax states
+ * are merged by log-sum-exp weight; needs gswa_workspace_bytes(
+ * GSWA_OP_FULL_DECODE) bytes of workspace (device, 16-byte aligned).
  */
 int full_decode(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                 const void *w_q, const void *w_k, void *k_cache, void *v_cache,
@@ -167,7 +174,9 @@ int64_t gswa_kv_cache_bytes(int n_global_layers, int n_window_layers, int window
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device: GSWA_OK, GSWA_ERR_TIMEOUT if a bounded wait inside a
- * kernel gave up since the last check, or GSWA_ERR_LAUNCH on a CUDA error.
+ * kernel gave up since the last check, GSWA_ERR_INVALID_ARG if a decode step
+ * found a position outside its cache (that sequence was skipped), or
+ * GSWA_ERR_LAUNCH on a CUDA error.
  */
 int gswa_check_status(void *stream);
 

@@ -74,3 +74,24 @@ def test_null_and_misaligned_pointers(L):
 def test_empty_problem_is_a_no_op(L):
     s = gca.make_shape(0, 64, 4, 1)
     assert _call_fwd(L, s, ptr=0) == 0
+
+
+def declared_arity():
+    """Parameter count of every function declared in include/*.h."""
+    out = {}
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(([^)]*)\)\s*;", text, flags=re.M):
+                params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+                out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_header(L):
+    """Every ctypes signature of the binding has the header's parameter count
+    (a short signature silently truncates the trailing stream handle)."""
+    arity = declared_arity()
+    for name, args in L._gswa_signatures.items():
+        assert arity[name] == len(args), (name, arity[name], len(args))

@@ -131,6 +131,16 @@ def decode_inputs(B, Hq, Hkv, D, cache_len, seed: int = 0, device="cpu", random_
     return dict(q=q, k=k, v=v, g=g, wq=wq, wk=wk, k_cache=kc, v_cache=vc)
 
 
+def fill_randn_bf16_(t: torch.Tensor, seed: int, chunk: int = 1 << 27) -> torch.Tensor:
+    """Fill a (possibly huge) bf16 tensor in place with N(0,1) values, slice by
+    slice, so no float32 copy of the whole tensor is ever held."""
+    flat = t.view(-1)
+    for i, part in enumerate(flat.split(chunk)):
+        g = _gen(seed * 1009 + i, t.device)
+        part.copy_(torch.randn(part.numel(), generator=g, device=t.device, dtype=torch.float32))
+    return t
+
+
 def sample_rows(T: int, n: int, seed: int = 0) -> torch.Tensor:
     """A seeded, sorted set of ``n`` distinct query positions in [0, T), always
     including the first and last position and the window edges 127/128."""
