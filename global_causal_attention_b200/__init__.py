@@ -158,6 +158,45 @@ def full_attn_fwd(q, k, v, wq, wk, *, rope_dims=42, rope_base=1e4, eps=1e-6, sca
     return y, lse
 
 
+def _bwd_outputs(q, k, gated):
+    torch = _torch()
+    D = q.shape[-1]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(k)
+    dg = torch.empty_like(q) if gated else None
+    dwq = torch.empty(D, dtype=torch.float32, device=q.device)
+    dwk = torch.empty(D, dtype=torch.float32, device=q.device)
+    return dq, dk, dv, dg, dwq, dwk
+
+
+def gswa_bwd(q, k, v, g, wq, wk, y, lse, dy, *, window=128, rope_dims=42, rope_base=1e4, eps=1e-6,
+             scale=None, workspace=None, stream=None):
+    """Backward of gswa_fwd given its y and lse and the upstream dy [B,T,Hq,D].
+    Returns (dq, dk, dv, dg) bf16 and (dw_q, dw_k) f32."""
+    _dev(q, k, v, g, wq, wk, y, lse, dy)
+    B, T, Hq, D = q.shape
+    s = make_shape(B, T, Hq, k.shape[2], D, window, rope_dims, rope_base, eps, scale)
+    dq, dk, dv, dg, dwq, dwk = _bwd_outputs(q, k, True)
+    ws, nb = _workspace(OP_GSWA_BWD, s, workspace, q.device)
+    _check(lib().gswa_bwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk), _ptr(y),
+                          _ptr(lse), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq), _ptr(dwk),
+                          _ptr(ws), nb, _stream(stream)), "gswa_bwd")
+    return dq, dk, dv, dg, dwq, dwk
+
+
+def full_attn_bwd(q, k, v, wq, wk, y, lse, dy, *, rope_dims=42, rope_base=1e4, eps=1e-6, scale=None,
+                  workspace=None, stream=None):
+    """Backward of full_attn_fwd.  Returns (dq, dk, dv) bf16 and (dw_q, dw_k) f32."""
+    _dev(q, k, v, wq, wk, y, lse, dy)
+    B, T, Hq, D = q.shape
+    s = make_shape(B, T, Hq, k.shape[2], D, 0, rope_dims, rope_base, eps, scale)
+    dq, dk, dv, _, dwq, dwk = _bwd_outputs(q, k, False)
+    ws, nb = _workspace(OP_FULL_BWD, s, workspace, q.device)
+    _check(lib().full_attn_bwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(y),
+                               _ptr(lse), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dwq), _ptr(dwk),
+                               _ptr(ws), nb, _stream(stream)), "full_attn_bwd")
+    return dq, dk, dv, dwq, dwk
+
+
 def gswa_qk_prep(x, w, *, rope_dims=42, rope_base=1e4, eps=1e-6, pos0=0, out=None, stream=None):
     """RMSNorm + partial RoPE of x [B, T, H, D] (bf16, cuda) at positions pos0 + t."""
     torch = _dev(x, w, out)

@@ -1,0 +1,1000 @@
+// bwd.cuh -- backward of the attention core (gated sliding window and full
+// causal), for sm_100a.
+//
+// The forward (ZGCM-1 §2.1, Figure 3 caption) is, per query row i of head h
+// (kv head h / 4), with q~ = RoPE(RMSNorm(q) w_q), k~ = RoPE(RMSNorm(k) w_k):
+//   S_ij = scale <q~_i, k~_j>,  P_ij = exp(S_ij - lse_i) over the visible j,
+//   A_i = sum_j P_ij v_j,  y_i = A_i ⊙ σ(g_i) (gated) or A_i (global layers).
+// Its gradients, given dy:
+//   dA = dy ⊙ σ(g),  dg = dy ⊙ y ⊙ (1 - σ(g))            (ungated: dA = dy)
+//   D_i = sum_d dA_i A_i = sum_d dy_i y_i
+//   dV_j = sum_i P_ij dA_i,  dP_ij = <dA_i, v_j>,  dS_ij = P_ij (dP_ij - D_i)
+//   dq~_i = scale sum_j dS_ij k~_j,  dk~_j = scale sum_i dS_ij q~_i
+//   dq = RMSNorm'(RoPE^T(dq~)), dk likewise, dw_q = sum dq^ ⊙ n_q, dw_k likewise.
+//
+// Kernels:
+//   bwd_prep     per row: D and lse log2 e into a row-ordered record, dA and
+//                dg (gated only)
+//   bwd_dq       query-stationary (M = 128 rows = 4 heads x 32 tokens): per key
+//                tile S = Q~K~^T and dP = dA V^T into TMEM; P from the
+//                forward's lse; dS (bf16, over S); dQ~ += dS K~ in TMEM;
+//                epilogue: RoPE^T and the RMSNorm backward against the raw q,
+//                per-warp dw_q partials
+//   bwd_dkdv     key-stationary (M = 128 keys of one kv head): per 64-row
+//                query chunk (16 tokens x 4 heads) S^T = K~Q~^T and
+//                dP^T = V dA^T; P^T and dS^T (bf16, over S^T and dP^T);
+//                dV += P^T dA and dK~ += dS^T Q~ in TMEM; epilogue: dv, and
+//                RoPE^T + RMSNorm backward against the raw k, dw_k partials
+//   dw_reduce    fixed-order sum of the weight-gradient partials
+// q~ and k~ come from qk_prep (workspace).  No atomics on global memory: the
+// results do not depend on scheduling.
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+#include "swa_fwd.cuh"
+
+namespace gswa {
+namespace bwd {
+
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr int kMaxGrid = 256;                 // bound on CTAs of the main kernels (partials sizing)
+constexpr uint32_t kHalfRowBytes = 128;       // one swizzled 64-dim half row
+
+// ------------------------------------------------------------------ pre-pass
+// Row record of the attention backward: {lse_i log2 e, D_i}, rows ordered
+// [B, Hkv, Tp, 4] (Tp = T rounded up to 32) so that the rows of one tile are
+// contiguous; rows t >= T hold {+inf, 0}, which makes their P exactly 0.
+struct PrepParams {
+    const __nv_bfloat16 *y, *dy, *g;   // g null: ungated
+    const float *lse;                  // [B, Hq, T]
+    __nv_bfloat16 *dA, *dg;            // [B, T, Hq, D]; null when ungated
+    float2 *ld;                        // [B, Hkv, Tp, 4]
+    long long rows;                    // B * Tp * Hq
+    int T, Tp, Hq;
+};
+
+constexpr int kPrepUnroll = 4;   // heads (rows) in flight per half-warp
+
+// A half-warp takes one token (b, t) at a time and walks its Hq rows four
+// heads at a time (one kv group, so the four records are contiguous); lane =
+// 8 dims, 16-byte accesses.  Tokens t >= T (the padding up to Tp) get
+// records only.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ PrepParams p)
+{
+    const int lane = threadIdx.x & 31, l16 = lane & 15;
+    // the two half-warps of a warp may take different branches: shuffle within one
+    const unsigned half_mask = 0xFFFFu << (lane & 16);
+    const unsigned nhw = gridDim.x * 16u;   // half-warps in the grid
+    const unsigned ntok = (unsigned)(p.rows / p.Hq);   // B * Tp
+    const int Hkv = p.Hq / 4;
+    for (unsigned bt = blockIdx.x * 16u + (threadIdx.x >> 4); bt < ntok; bt += nhw) {
+        const unsigned b = bt / (unsigned)p.Tp;
+        const int t = (int)(bt - b * (unsigned)p.Tp);
+        float2 *rec = p.ld + ((long long)b * Hkv * p.Tp + t) * 4;   // + (kvh Tp) 4 + h % 4
+        if (t >= p.T) {
+            // padded token: P = 0 for every key
+            if (l16 < Hkv * 4)
+                for (int h = l16; h < p.Hq; h += 16)
+                    rec[(long long)(h >> 2) * p.Tp * 4 + (h & 3)] = make_float2(INFINITY, 0.f);
+            continue;
+        }
+        const long long row0 = ((long long)b * p.T + t) * p.Hq;
+        for (int h0 = 0; h0 < p.Hq; h0 += kPrepUnroll) {
+            uint4 yv[kPrepUnroll], dv[kPrepUnroll], gv[kPrepUnroll];
+#pragma unroll
+            for (int u = 0; u < kPrepUnroll; ++u) {
+                const long long off = (row0 + h0 + u) * kD + 8 * l16;
+                yv[u] = *reinterpret_cast<const uint4 *>(p.y + off);
+                dv[u] = *reinterpret_cast<const uint4 *>(p.dy + off);
+                if (p.g != nullptr) gv[u] = *reinterpret_cast<const uint4 *>(p.g + off);
+            }
+            float dsum[kPrepUnroll];
+#pragma unroll
+            for (int u = 0; u < kPrepUnroll; ++u) {
+                const uint32_t ya[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
+                const uint32_t da[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 yy = unpack_bf16(ya[e]), dd = unpack_bf16(da[e]);
+                    s = fmaf(dd.x, yy.x, fmaf(dd.y, yy.y, s));
+                }
+                dsum[u] = s;
+                if (p.g != nullptr) {
+                    const uint32_t ga[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+                    uint32_t oa[4], og[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 gg = unpack_bf16(ga[e]), yy = unpack_bf16(ya[e]), dd = unpack_bf16(da[e]);
+                        const float s0 = 1.f / (1.f + __expf(-gg.x)), s1 = 1.f / (1.f + __expf(-gg.y));
+                        oa[e] = pack_bf16(dd.x * s0, dd.y * s1);
+                        og[e] = pack_bf16(dd.x * yy.x * (1.f - s0), dd.y * yy.y * (1.f - s1));
+                    }
+                    const long long off = (row0 + h0 + u) * kD + 8 * l16;
+                    *reinterpret_cast<uint4 *>(p.dA + off) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                    *reinterpret_cast<uint4 *>(p.dg + off) = make_uint4(og[0], og[1], og[2], og[3]);
+                }
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+                for (int u = 0; u < kPrepUnroll; ++u) dsum[u] += __shfl_xor_sync(half_mask, dsum[u], o);
+            if (l16 < kPrepUnroll) {
+                // lane u of the half-warp writes the record of head h0 + u
+                float dv_u = dsum[0];
+#pragma unroll
+                for (int u = 1; u < kPrepUnroll; ++u) dv_u = (l16 == u) ? dsum[u] : dv_u;
+                const int h = h0 + l16;
+                rec[(long long)(h >> 2) * p.Tp * 4 + (h & 3)] =
+                    make_float2(p.lse[((long long)b * p.Hq + h) * p.T + t] * 1.4426950408889634f, dv_u);
+            }
+        }
+    }
+}
+
+// dw[d] = sum over the partials, in a fixed order (deterministic): thread
+// (slice s, dim d) sums partials s, s + 8, ... in order, then the 8 slice
+// sums are added in slice order.
+constexpr int kReduceSlices = 8;
+__global__ void __launch_bounds__(kD * kReduceSlices) dw_reduce_kernel(const float *part, int nparts, float *dw)
+{
+    __shared__ float acc[kReduceSlices][kD];
+    const int d = threadIdx.x & (kD - 1), sl = threadIdx.x / kD;
+    float s0 = 0.f, s1 = 0.f;
+    int i = sl;
+    for (; i + kReduceSlices < nparts; i += 2 * kReduceSlices) {
+        s0 += part[(long long)i * kD + d];
+        s1 += part[(long long)(i + kReduceSlices) * kD + d];
+    }
+    if (i < nparts) s0 += part[(long long)i * kD + d];
+    acc[sl][d] = s0 + s1;
+    __syncthreads();
+    if (sl == 0) {
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < kReduceSlices; ++k) s += acc[k][d];
+        dw[d] = s;
+    }
+}
+
+// --------------------------------------------------------- shared machinery
+struct Params {
+    int B, T, Tp, Hq, Hkv, window;   // window: sliding-window width (ignored by the full kernels)
+    int nq;                          // query blocks of 32 tokens
+    int nkt;                         // key tiles (dq: of kN keys; dkdv: of 128 keys)
+    long long units;
+    float eps, sl2, scale;           // sl2 = scale log2 e
+    const float2 *ld;                // row records (see PrepParams)
+    const __nv_bfloat16 *x;          // raw q (dq kernel) or raw k (dkdv kernel)
+    const __nv_bfloat16 *w;          // w_q or w_k
+    __nv_bfloat16 *dx;               // dq or dk
+    __nv_bfloat16 *dv;               // dkdv kernel: dv
+    float *dw_part;                  // [gridDim.x * 4][128] per-warp partial weight gradients
+    double theta[64];
+};
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > 200000000ull) break;
+}
+
+// k-th unit of this CTA in a longest-first "snake" order over `units`
+// (unit u of the order goes to CTA u mod 2G or 2G - 1 - u mod 2G).
+__device__ __forceinline__ long long snake_unit(int k)
+{
+    const long long G = gridDim.x, c = blockIdx.x;
+    return (k & 1) ? ((long long)(k + 1) * G - 1 - c) : ((long long)k * G + c);
+}
+
+__device__ __forceinline__ int snake_count(long long units)
+{
+    const long long G = gridDim.x, c = blockIdx.x;
+    const long long full = units / (2 * G), rem = units - full * 2 * G;
+    return (int)(2 * full + (c < rem ? 1 : 0) + (2 * G - 1 - c < rem ? 1 : 0));
+}
+
+// Warp reduce-scatter: on return, lane l holds the warp-wide sum of a[l].
+__device__ __forceinline__ float warp_reduce_scatter32(float (&a)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+            const float send = upper ? a[i] : a[i + k];
+            const float keep = upper ? a[i + k] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+    return a[0];
+}
+
+// Rotate one TMEM row of 128 f32 gradients back through RoPE_pos^T, in place:
+//   (g_p, g_{p+R/2}) <- (g_p c + g_{p+R/2} s, g_{p+R/2} c - g_p s).
+template <int R>
+__device__ __forceinline__ void rope_back_tmem(uint32_t trow, int pos, const double *theta)
+{
+    constexpr int H = R / 2;
+    if constexpr (R > 0) {
+        constexpr int kRounds = (R == 128) ? 2 : 1;
+        static_assert(R <= 64 || R == 128, "rotary width");
+#pragma unroll
+        for (int rd = 0; rd < kRounds; ++rd) {
+            // R <= 64: dims 0..63 (chunks 0, 1); R = 128: chunk rd pairs with chunk rd + 2
+            const uint32_t ca = trow + 32 * rd, cb = trow + ((R == 128) ? 32 * (rd + 2) : 32);
+            uint32_t a[32], b[32];
+            tmem_ld32(ca, a);
+            tmem_ld32(cb, b);
+            tmem_wait_ld();
+            if constexpr (R == 128) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float c, s;
+                    swa::rope_cs(theta[32 * rd + e], pos, c, s);
+                    const float g1 = __uint_as_float(a[e]), g2 = __uint_as_float(b[e]);
+                    a[e] = __float_as_uint(g1 * c + g2 * s);
+                    b[e] = __float_as_uint(g2 * c - g1 * s);
+                }
+            } else {
+                float u[64];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    u[e] = __uint_as_float(a[e]);
+                    u[32 + e] = __uint_as_float(b[e]);
+                }
+#pragma unroll
+                for (int pp = 0; pp < H; ++pp) {
+                    float c, s;
+                    swa::rope_cs(theta[pp], pos, c, s);
+                    const float g1 = u[pp], g2 = u[pp + H];
+                    u[pp] = g1 * c + g2 * s;
+                    u[pp + H] = g2 * c - g1 * s;
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    a[e] = __float_as_uint(u[e]);
+                    b[e] = __float_as_uint(u[32 + e]);
+                }
+            }
+            uint32_t lo[16], hi[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                lo[e] = a[e];
+                hi[e] = a[16 + e];
+            }
+            tmem_st16(ca, lo);
+            tmem_st16(ca + 16, hi);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                lo[e] = b[e];
+                hi[e] = b[16 + e];
+            }
+            tmem_st16(cb, lo);
+            tmem_st16(cb + 16, hi);
+        }
+        tmem_wait_st();
+    }
+}
+
+// RoPE^T and RMSNorm backward of one row.  The gradient w.r.t. the prepared
+// row is `gscale` times the f32 row at TMEM address `trow` (this thread's
+// lane); x is the raw row (bf16, global), pos its position:
+//   du = RoPE_pos^T(g);  r = (mean x^2 + eps)^-1/2;  n = x r;
+//   dx = r (w ⊙ du - n mean(w ⊙ du ⊙ n));  dw += du ⊙ n.
+// Every lane of the warp must call it (TMEM loads are warp-wide); a lane
+// with valid == false contributes nothing and writes nothing.  dwacc[c] of
+// lane l accumulates dim 32 c + l of the warp's dw sum.
+template <int R>
+__device__ __forceinline__ void norm_rope_backward(uint32_t trow, float gscale, const __nv_bfloat16 *xrow,
+                                                   bool valid, const float *w, float eps, int pos,
+                                                   const double *theta, __nv_bfloat16 *dxrow, float (&dwacc)[4])
+{
+    rope_back_tmem<R>(trow, pos, theta);
+    const float gs = valid ? gscale : 0.f;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(xrow);
+    // pass 1: sum x^2 and sum w g x
+    float ss = 0.f, wgx = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + 32 * c, v);
+        uint4 xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = xr[4 * c + q];
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t x4[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int d = 32 * c + 8 * q + 2 * e;
+                const float2 f = unpack_bf16(x4[e]);
+                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                wgx = fmaf(w[d] * __uint_as_float(v[8 * q + 2 * e]), f.x,
+                           fmaf(w[d + 1] * __uint_as_float(v[8 * q + 2 * e + 1]), f.y, wgx));
+            }
+        }
+    }
+    const float r = rsqrtf(ss * (1.0f / kD) + eps);
+    const float m = gs * r * wgx * (1.0f / kD);   // mean(w du n)
+    // pass 2: dx and dw
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + 32 * c, v);
+        uint4 xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = xr[4 * c + q];
+        tmem_wait_ld();
+        float pw[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t x4[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int d = 32 * c + 8 * q + 2 * e;
+                const float2 f = unpack_bf16(x4[e]);
+                const float du0 = gs * __uint_as_float(v[8 * q + 2 * e]);
+                const float du1 = gs * __uint_as_float(v[8 * q + 2 * e + 1]);
+                const float n0 = f.x * r, n1 = f.y * r;
+                o4[e] = pack_bf16(r * fmaf(w[d], du0, -n0 * m), r * fmaf(w[d + 1], du1, -n1 * m));
+                pw[8 * q + 2 * e] = du0 * n0;
+                pw[8 * q + 2 * e + 1] = du1 * n1;
+            }
+            if (valid) reinterpret_cast<uint4 *>(dxrow)[4 * c + q] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        dwacc[c] += warp_reduce_scatter32(pw);
+    }
+}
+
+// ============================================================== dq kernel
+template <bool kSwa>
+struct DqCfg {
+    static constexpr int kN = kSwa ? 160 : 64;       // keys per tile (sliding window: the unit's span)
+    static constexpr int kNBuf = kSwa ? 1 : 2;       // S/dP buffers in TMEM
+    static constexpr int kStages = kSwa ? 2 : 4;     // K~/V stages in shared memory
+    static constexpr uint32_t kQHalf = 128 * kHalfRowBytes;   // 16 KiB
+    static constexpr uint32_t kQTile = 2 * kQHalf;
+    static constexpr uint32_t kKHalf = kN * kHalfRowBytes;
+    static constexpr uint32_t kKTile = 2 * kKHalf;
+    static constexpr uint32_t kOffQ = 0;
+    static constexpr uint32_t kOffA = kOffQ + kQTile;
+    static constexpr uint32_t kOffK = kOffA + kQTile;
+    static constexpr uint32_t kOffV = kOffK + kStages * kKTile;
+    static constexpr uint32_t kOffW = kOffV + kStages * kKTile;   // f32[128]
+    static constexpr uint32_t kOffBar = kOffW + 512;
+    static constexpr int kNumBars = 24;
+    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+    static constexpr uint32_t kColDQ = kNBuf * 2 * kN;
+    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    static_assert(kColDQ + 128 <= 512, "TMEM budget");
+    // barrier indices
+    static constexpr int BQ_FULL = 0, BQ_EMPTY = 1, BKV_FULL = 2, BKV_EMPTY = BKV_FULL + kStages,
+                         BS_FULL = BKV_EMPTY + kStages, BDS_READY = BS_FULL + kNBuf,
+                         BS_FREE = BDS_READY + kNBuf, BACC_FULL = BS_FREE + kNBuf, BACC_FREE = BACC_FULL + 1,
+                         B_DRAIN = BACC_FREE + 1;
+    static_assert(B_DRAIN < kNumBars, "barrier count");
+};
+
+struct QUnit {
+    int b, kvh, qb, n;   // n: key tiles of the unit
+};
+
+template <bool kSwa>
+__device__ __forceinline__ bool dq_unit_at(const Params &p, int k, QUnit &x)
+{
+    const long long u = snake_unit(k);
+    if (u >= p.units) return false;
+    const long long per = (long long)p.B * p.Hkv;
+    x.qb = p.nq - 1 - (int)(u / per);
+    const long long strip = u % per;
+    x.b = (int)(strip / p.Hkv);
+    x.kvh = (int)(strip % p.Hkv);
+    x.n = kSwa ? 1 : min(p.nkt, (32 * x.qb + 31) / DqCfg<kSwa>::kN + 1);
+    return true;
+}
+
+// first key of tile j of a unit
+template <bool kSwa>
+__device__ __forceinline__ int dq_tile_key0(const QUnit &x, int j)
+{
+    return kSwa ? 32 * x.qb - 128 : j * DqCfg<kSwa>::kN;
+}
+
+template <bool kSwa>
+struct DqWalk {
+    int k = 0, j = 0;
+    QUnit x;
+    bool valid = false;
+    __device__ __forceinline__ void init(const Params &p) { k = 0; j = 0; valid = dq_unit_at<kSwa>(p, 0, x); }
+    __device__ __forceinline__ bool last() const { return j == x.n - 1; }
+    __device__ __forceinline__ void next(const Params &p)
+    {
+        if (++j == x.n) {
+            j = 0;
+            ++k;
+            valid = dq_unit_at<kSwa>(p, k, x);
+        }
+    }
+};
+
+template <int R, bool kSwa>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
+              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ Params p)
+{
+    using C = DqCfg<kSwa>;
+    constexpr int kN = C::kN, kNBuf = C::kNBuf, kStages = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    Abort ab{reinterpret_cast<volatile int *>(smem + C::kOffAbort)};
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * (uint32_t)i; };
+    const int nunits = snake_count(p.units);
+
+    if (tid == 0) {
+        *ab.flag = 0;
+        mbar_init(bar(C::BQ_FULL), 1);
+        mbar_init(bar(C::BQ_EMPTY), 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(bar(C::BKV_FULL + i), 1);
+            mbar_init(bar(C::BKV_EMPTY + i), 1);
+        }
+        for (int i = 0; i < kNBuf; ++i) {
+            mbar_init(bar(C::BS_FULL + i), 1);
+            mbar_init(bar(C::BDS_READY + i), 4);
+            mbar_init(bar(C::BS_FREE + i), 1);
+        }
+        mbar_init(bar(C::BACC_FULL), 1);
+        mbar_init(bar(C::BACC_FREE), 4);
+        mbar_init(bar(C::B_DRAIN), 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (tid < 128) reinterpret_cast<float *>(smem + C::kOffW)[tid] = __bfloat162float(p.w[tid]);
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            int g = 0, k = 0;
+            QUnit x;
+            bool ok = true;
+            for (; k < nunits && ok; ++k) {
+                dq_unit_at<kSwa>(p, k, x);
+                ok = mbar_wait(bar(C::BQ_EMPTY), (k & 1) ^ 1u, ab);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::BQ_FULL), 2 * C::kQTile);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_4d(sbase + C::kOffQ + h * C::kQHalf, &tm_q, bar(C::BQ_FULL), h * 64, x.kvh * 4,
+                                x.qb * 32, x.b);
+                    tma_load_4d(sbase + C::kOffA + h * C::kQHalf, &tm_a, bar(C::BQ_FULL), h * 64, x.kvh * 4,
+                                x.qb * 32, x.b);
+                }
+                for (int j = 0; j < x.n && ok; ++j, ++g) {
+                    const int st = g % kStages;
+                    ok = mbar_wait(bar(C::BKV_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(bar(C::BKV_FULL + st), 2 * C::kKTile);
+                    const int key0 = dq_tile_key0<kSwa>(x, j);
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_4d(sbase + C::kOffK + st * C::kKTile + h * C::kKHalf, &tm_k,
+                                    bar(C::BKV_FULL + st), h * 64, x.kvh, key0, x.b);
+                        tma_load_4d(sbase + C::kOffV + st * C::kKTile + h * C::kKHalf, &tm_v,
+                                    bar(C::BKV_FULL + st), h * 64, x.kvh, key0, x.b);
+                    }
+                }
+            }
+            // no copy may still be landing when the CTA exits
+            for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
+                drain_wait(bar(C::BKV_FULL + i % kStages), (i / kStages) & 1);
+            if (k > 0) drain_wait(bar(C::BQ_FULL), (k - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, kN, 0, 0);
+            const uint32_t idesc_dq = idesc_bf16_f32(128, 128, 0, 1);
+            DqWalk<kSwa> ws, wd;
+            ws.init(p);
+            wd.init(p);
+            int ns = 0, nd = 0;
+            uint64_t t_last = globaltimer();
+            while (wd.valid) {
+                bool progressed = false;
+                if (ws.valid && ns < nd + kNBuf && mbar_test(bar(C::BQ_FULL), ws.k & 1) &&
+                    mbar_test(bar(C::BKV_FULL + ns % kStages), (ns / kStages) & 1) &&
+                    mbar_test(bar(C::BS_FREE + ns % kNBuf), ((ns / kNBuf) & 1) ^ 1u)) {
+                    tc_fence_after();
+                    const uint32_t dS = tmem + (ns % kNBuf) * 2 * kN;
+                    const uint32_t ks = sbase + C::kOffK + (ns % kStages) * C::kKTile;
+                    const uint32_t vs = sbase + C::kOffV + (ns % kStages) * C::kKTile;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t oq = (kk >> 2) * C::kQHalf + (kk & 3) * 32;
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        mma_ss(dS, smem_desc_sw128(sbase + C::kOffQ + oq, 16, 1024),
+                               smem_desc_sw128(ks + ok_, 16, 1024), idesc_s, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t oq = (kk >> 2) * C::kQHalf + (kk & 3) * 32;
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        mma_ss(dS + kN, smem_desc_sw128(sbase + C::kOffA + oq, 16, 1024),
+                               smem_desc_sw128(vs + ok_, 16, 1024), idesc_s, kk > 0);
+                    }
+                    mma_commit(bar(C::BS_FULL + ns % kNBuf));
+                    if (ws.last()) mma_commit(bar(C::BQ_EMPTY));
+                    ws.next(p);
+                    ++ns;
+                    progressed = true;
+                }
+                if (nd < ns && mbar_test(bar(C::BDS_READY + nd % kNBuf), (nd / kNBuf) & 1) &&
+                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
+                    tc_fence_after();
+                    const uint32_t ks = sbase + C::kOffK + (nd % kStages) * C::kKTile;
+                    const uint32_t da = tmem + (nd % kNBuf) * 2 * kN;
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk)
+                        mma_ts(tmem + C::kColDQ, da + kk * 8, smem_desc_sw128(ks + kk * 16 * 128, C::kKHalf, 1024),
+                               idesc_dq, (wd.j > 0 || kk > 0));
+                    mma_commit(bar(C::BKV_EMPTY + nd % kStages));
+                    mma_commit(bar(C::BS_FREE + nd % kNBuf));
+                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
+                    wd.next(p);
+                    ++nd;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = globaltimer();
+                } else {
+                    if (ab.raised()) break;
+                    if (globaltimer() - t_last > kWaitLimitNs) {
+                        ab.raise(kStatusTimeout);
+                        break;
+                    }
+                }
+            }
+            mma_commit(bar(C::B_DRAIN));
+            drain_wait(bar(C::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================= dS = P (dP - D)
+        const int r = tid - 128;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const int W = kSwa ? p.window : 0;
+        bool ok = true;
+        int g = 0;
+        QUnit x;
+        for (int k = 0; k < nunits && ok; ++k) {
+            dq_unit_at<kSwa>(p, k, x);
+            const int i = x.qb * 32 + (r >> 2);
+            const float2 rec = p.ld[(((long long)x.b * p.Hkv + x.kvh) * p.Tp + x.qb * 32) * 4 + r];
+            const float lse2 = rec.x, Dv = rec.y;
+            for (int j = 0; j < x.n && ok; ++j, ++g) {
+                const int bb = g % kNBuf;
+                ok = warp_wait(bar(C::BS_FULL + bb), (g / kNBuf) & 1, ab);
+                if (!ok) break;
+                tc_fence_after();
+                const int key0 = dq_tile_key0<kSwa>(x, j);
+                const int hi = i - key0;                                   // visible columns: lo <= c <= hi
+                const int lo = kSwa ? max(-key0, hi - W + 1) : 0;
+                const uint32_t ts = tmem + lane_base + bb * 2 * kN;
+#pragma unroll 1
+                for (int c = 0; c < kN / 32; ++c) {
+                    uint32_t s[32], d[32], pk[16];
+                    tmem_ld32(ts + 32 * c, s);
+                    tmem_ld32(ts + kN + 32 * c, d);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int col = 32 * c + e;
+                        float p0 = ex2(fmaf(__uint_as_float(s[e]), p.sl2, -lse2));
+                        float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), p.sl2, -lse2));
+                        p0 = (col >= lo && col <= hi) ? p0 : 0.f;
+                        p1 = (col + 1 >= lo && col + 1 <= hi) ? p1 : 0.f;
+                        pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(d[e]) - Dv),
+                                               p1 * (__uint_as_float(d[e + 1]) - Dv));
+                    }
+                    tmem_st16(ts + 16 * c, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BDS_READY + bb));
+            }
+        }
+    } else if (warp >= 8) {
+        // ================================================= epilogue: dq, dw_q
+        const int r = tid - 256;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
+        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
+        bool ok = true;
+        QUnit x;
+        for (int k = 0; k < nunits && ok; ++k) {
+            dq_unit_at<kSwa>(p, k, x);
+            ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
+            if (!ok) break;
+            tc_fence_after();
+            const int i = x.qb * 32 + (r >> 2);
+            const bool valid = i < p.T;
+            const long long off = valid ? (((long long)x.b * p.T + i) * p.Hq + x.kvh * 4 + (r & 3)) * kD : 0;
+            norm_rope_backward<R>(tmem + lane_base + C::kColDQ, p.scale, p.x + off, valid, w, p.eps, i, p.theta,
+                                  p.dx + off, dwacc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::BACC_FREE));
+        }
+        float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================ dk/dv kernel
+struct KvCfg {
+    static constexpr int kM = 64;                    // query rows per chunk (16 tokens x 4 heads)
+    static constexpr int kChTok = 16;
+    static constexpr int kStages = 4;
+    static constexpr uint32_t kKHalf = 128 * kHalfRowBytes;   // 16 KiB
+    static constexpr uint32_t kKTile = 2 * kKHalf;
+    static constexpr uint32_t kCHalf = kM * kHalfRowBytes;    // 8 KiB
+    static constexpr uint32_t kCTile = 2 * kCHalf;
+    static constexpr uint32_t kStageBytes = 2 * kCTile + 1024;   // Q~ chunk, dA chunk, records (512 B)
+    static constexpr uint32_t kOffK = 0;
+    static constexpr uint32_t kOffV = kOffK + kKTile;
+    static constexpr uint32_t kOffCh = kOffV + kKTile;
+    static constexpr uint32_t kOffW = kOffCh + kStages * kStageBytes;
+    static constexpr uint32_t kOffBar = kOffW + 512;
+    static constexpr int kNumBars = 24;
+    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+    static constexpr uint32_t kColDV = 256, kColDK = 384;
+    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    static constexpr int BKV_FULL = 0, BKV_EMPTY = 1, BCH_FULL = 2, BCH_EMPTY = BCH_FULL + kStages,
+                         BS_FULL = BCH_EMPTY + kStages, BP_READY = BS_FULL + 2, BS_FREE = BP_READY + 2,
+                         BACC_FULL = BS_FREE + 2, BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1;
+    static_assert(B_DRAIN < kNumBars, "barrier count");
+};
+
+struct KUnit {
+    int b, kvh, kt, n;   // n: query chunks of the unit
+};
+
+template <bool kSwa>
+__device__ __forceinline__ bool kv_unit_at(const Params &p, int k, KUnit &x)
+{
+    const long long u = snake_unit(k);
+    if (u >= p.units) return false;
+    const long long per = (long long)p.B * p.Hkv;
+    x.kt = (int)(u / per);
+    const long long strip = u % per;
+    x.b = (int)(strip / p.Hkv);
+    x.kvh = (int)(strip % p.Hkv);
+    const int k0 = 128 * x.kt;
+    // queries that see keys [k0, k0 + 128): i in [k0, k0 + 127 + W - 1] (sliding) or [k0, T)
+    const int span = kSwa ? min(127 + p.window, p.T - k0) : p.T - k0;
+    x.n = (span + KvCfg::kChTok - 1) / KvCfg::kChTok;
+    return true;
+}
+
+template <bool kSwa>
+struct KvWalk {
+    int k = 0, j = 0;
+    KUnit x;
+    bool valid = false;
+    __device__ __forceinline__ void init(const Params &p) { k = 0; j = 0; valid = kv_unit_at<kSwa>(p, 0, x); }
+    __device__ __forceinline__ bool last() const { return j == x.n - 1; }
+    __device__ __forceinline__ void next(const Params &p)
+    {
+        if (++j == x.n) {
+            j = 0;
+            ++k;
+            valid = kv_unit_at<kSwa>(p, k, x);
+        }
+    }
+};
+
+template <int R, bool kSwa>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
+                const __grid_constant__ Params p)
+{
+    using C = KvCfg;
+    constexpr int kM = C::kM, kStages = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    Abort ab{reinterpret_cast<volatile int *>(smem + C::kOffAbort)};
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * (uint32_t)i; };
+    auto stage = [&](int st) -> uint32_t { return sbase + C::kOffCh + (uint32_t)st * C::kStageBytes; };
+    const int nunits = snake_count(p.units);
+
+    if (tid == 0) {
+        *ab.flag = 0;
+        mbar_init(bar(C::BKV_FULL), 1);
+        mbar_init(bar(C::BKV_EMPTY), 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(bar(C::BCH_FULL + i), 1);
+            mbar_init(bar(C::BCH_EMPTY + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::BS_FULL + i), 1);
+            mbar_init(bar(C::BP_READY + i), 4);
+            mbar_init(bar(C::BS_FREE + i), 1);
+        }
+        mbar_init(bar(C::BACC_FULL), 1);
+        mbar_init(bar(C::BACC_FREE), 4);
+        mbar_init(bar(C::B_DRAIN), 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_a);
+    }
+    if (tid < 128) reinterpret_cast<float *>(smem + C::kOffW)[tid] = __bfloat162float(p.w[tid]);
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            int g = 0, k = 0;
+            KUnit x;
+            bool ok = true;
+            for (; k < nunits && ok; ++k) {
+                kv_unit_at<kSwa>(p, k, x);
+                ok = mbar_wait(bar(C::BKV_EMPTY), (k & 1) ^ 1u, ab);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::BKV_FULL), 2 * C::kKTile);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_4d(sbase + C::kOffK + h * C::kKHalf, &tm_k, bar(C::BKV_FULL), h * 64, x.kvh,
+                                128 * x.kt, x.b);
+                    tma_load_4d(sbase + C::kOffV + h * C::kKHalf, &tm_v, bar(C::BKV_FULL), h * 64, x.kvh,
+                                128 * x.kt, x.b);
+                }
+                for (int j = 0; j < x.n && ok; ++j, ++g) {
+                    const int st = g % kStages;
+                    ok = mbar_wait(bar(C::BCH_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
+                    if (!ok) break;
+                    const int t0 = 128 * x.kt + C::kChTok * j;
+                    mbar_arrive_expect_tx(bar(C::BCH_FULL + st), 2 * C::kCTile + kM * 8);
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_4d(stage(st) + h * C::kCHalf, &tm_q, bar(C::BCH_FULL + st), h * 64, x.kvh * 4, t0,
+                                    x.b);
+                        tma_load_4d(stage(st) + C::kCTile + h * C::kCHalf, &tm_a, bar(C::BCH_FULL + st), h * 64,
+                                    x.kvh * 4, t0, x.b);
+                    }
+                    bulk_load(stage(st) + 2 * C::kCTile, p.ld + (((long long)x.b * p.Hkv + x.kvh) * p.Tp + t0) * 4,
+                              kM * 8, bar(C::BCH_FULL + st));
+                }
+            }
+            for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
+                drain_wait(bar(C::BCH_FULL + i % kStages), (i / kStages) & 1);
+            if (k > 0) drain_wait(bar(C::BKV_FULL), (k - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, kM, 0, 0);
+            const uint32_t idesc_acc = idesc_bf16_f32(128, 128, 0, 1);
+            KvWalk<kSwa> ws, wd;
+            ws.init(p);
+            wd.init(p);
+            int ns = 0, nd = 0;
+            uint64_t t_last = globaltimer();
+            while (wd.valid) {
+                bool progressed = false;
+                if (ws.valid && ns < nd + 2 && mbar_test(bar(C::BKV_FULL), ws.k & 1) &&
+                    mbar_test(bar(C::BCH_FULL + ns % kStages), (ns / kStages) & 1) &&
+                    mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
+                    tc_fence_after();
+                    const uint32_t dS = tmem + (ns & 1) * 128;
+                    const uint32_t qs = stage(ns % kStages), as = qs + C::kCTile;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        const uint32_t oc = (kk >> 2) * C::kCHalf + (kk & 3) * 32;
+                        mma_ss(dS, smem_desc_sw128(sbase + C::kOffK + ok_, 16, 1024),
+                               smem_desc_sw128(qs + oc, 16, 1024), idesc_s, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        const uint32_t oc = (kk >> 2) * C::kCHalf + (kk & 3) * 32;
+                        mma_ss(dS + kM, smem_desc_sw128(sbase + C::kOffV + ok_, 16, 1024),
+                               smem_desc_sw128(as + oc, 16, 1024), idesc_s, kk > 0);
+                    }
+                    mma_commit(bar(C::BS_FULL + (ns & 1)));
+                    if (ws.last()) mma_commit(bar(C::BKV_EMPTY));
+                    ws.next(p);
+                    ++ns;
+                    progressed = true;
+                }
+                if (nd < ns && mbar_test(bar(C::BP_READY + (nd & 1)), (nd >> 1) & 1) &&
+                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
+                    tc_fence_after();
+                    const uint32_t pt = tmem + (nd & 1) * 128;
+                    const uint32_t qs = stage(nd % kStages), as = qs + C::kCTile;
+#pragma unroll
+                    for (int kk = 0; kk < kM / 16; ++kk)
+                        mma_ts(tmem + C::kColDV, pt + kk * 8, smem_desc_sw128(as + kk * 16 * 128, C::kCHalf, 1024),
+                               idesc_acc, (wd.j > 0 || kk > 0));
+#pragma unroll
+                    for (int kk = 0; kk < kM / 16; ++kk)
+                        mma_ts(tmem + C::kColDK, pt + kM + kk * 8,
+                               smem_desc_sw128(qs + kk * 16 * 128, C::kCHalf, 1024), idesc_acc, (wd.j > 0 || kk > 0));
+                    mma_commit(bar(C::BCH_EMPTY + nd % kStages));
+                    mma_commit(bar(C::BS_FREE + (nd & 1)));
+                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
+                    wd.next(p);
+                    ++nd;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = globaltimer();
+                } else {
+                    if (ab.raised()) break;
+                    if (globaltimer() - t_last > kWaitLimitNs) {
+                        ab.raise(kStatusTimeout);
+                        break;
+                    }
+                }
+            }
+            mma_commit(bar(C::B_DRAIN));
+            drain_wait(bar(C::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================= P^T, dS^T
+        const int r = tid - 128;   // key of the tile
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const int W = kSwa ? p.window : (1 << 30);
+        bool ok = true;
+        int g = 0;
+        KUnit x;
+        for (int k = 0; k < nunits && ok; ++k) {
+            kv_unit_at<kSwa>(p, k, x);
+            const int jkey = 128 * x.kt + r;
+            for (int j = 0; j < x.n && ok; ++j, ++g) {
+                const int bb = g & 1, st = g % kStages;
+                ok = warp_wait(bar(C::BS_FULL + bb), (g >> 1) & 1, ab);
+                // the stage's records: its load completed before the MMA read the stage
+                if (ok) ok = warp_wait(bar(C::BCH_FULL + st), (g / kStages) & 1, ab);
+                if (!ok) break;
+                tc_fence_after();
+                const int t0 = 128 * x.kt + C::kChTok * j;
+                const int lo = jkey - t0, hi = jkey - t0 + W - 1;   // visible chunk tokens
+                const uint32_t ts = tmem + lane_base + bb * 128;
+                const uint32_t rec = stage(st) + 2 * C::kCTile;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t s[32], d[32], pk[16], dk[16];
+                    tmem_ld32(ts + 32 * hf, s);
+                    tmem_ld32(ts + kM + 32 * hf, d);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        // records of rows 32 hf + e .. + 3 (one token, four heads)
+                        const uint4 ra = lds128(rec + (32 * hf + e) * 8);
+                        const uint4 rb = lds128(rec + (32 * hf + e + 2) * 8);
+                        const float l2[4] = {__uint_as_float(ra.x), __uint_as_float(ra.z), __uint_as_float(rb.x),
+                                             __uint_as_float(rb.z)};
+                        const float dv[4] = {__uint_as_float(ra.y), __uint_as_float(ra.w), __uint_as_float(rb.y),
+                                             __uint_as_float(rb.w)};
+                        const int tok = (32 * hf + e) >> 2;
+                        const bool vis = tok >= lo && tok <= hi;
+                        float pp[4], ds[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            pp[q] = vis ? ex2(fmaf(__uint_as_float(s[e + q]), p.sl2, -l2[q])) : 0.f;
+                            ds[q] = pp[q] * (__uint_as_float(d[e + q]) - dv[q]);
+                        }
+                        pk[e >> 1] = pack_bf16(pp[0], pp[1]);
+                        pk[(e >> 1) + 1] = pack_bf16(pp[2], pp[3]);
+                        dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                        dk[(e >> 1) + 1] = pack_bf16(ds[2], ds[3]);
+                    }
+                    tmem_st16(ts + 16 * hf, pk);
+                    tmem_st16(ts + kM + 16 * hf, dk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BP_READY + bb));
+            }
+        }
+    } else if (warp >= 8) {
+        // ================================================= epilogue: dv, dk, dw_k
+        const int r = tid - 256;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
+        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
+        bool ok = true;
+        KUnit x;
+        for (int k = 0; k < nunits && ok; ++k) {
+            kv_unit_at<kSwa>(p, k, x);
+            ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
+            if (!ok) break;
+            tc_fence_after();
+            const int jkey = 128 * x.kt + r;
+            const bool valid = jkey < p.T;
+            const long long off = valid ? (((long long)x.b * p.T + jkey) * p.Hkv + x.kvh) * kD : 0;
+            // dv = sum_i P_ij dA_i
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + C::kColDV + 32 * c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 o = make_uint4(
+                        pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1])),
+                        pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                        pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                        pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+                    if (valid) reinterpret_cast<uint4 *>(p.dv + off)[4 * c + q] = o;
+                }
+            }
+            norm_rope_backward<R>(tmem + lane_base + C::kColDK, p.scale, p.x + off, valid, w, p.eps, jkey,
+                                  p.theta, p.dx + off, dwacc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::BACC_FREE));
+        }
+        float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace bwd
+}  // namespace gswa

@@ -17,6 +17,7 @@
 #include "qk_prep.cuh"
 #include "full_fwd.cuh"
 #include "decode.cuh"
+#include "bwd.cuh"
 
 namespace {
 
@@ -42,6 +43,16 @@ bool set_smem(K kernel, uint32_t bytes)
 {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
            cudaSuccess;
+}
+
+template <int R>
+bool set_bwd_smem()
+{
+    using namespace gswa::bwd;
+    return set_smem(bwd_dq_kernel<R, true>, DqCfg<true>::kSmemBytes) ||
+           set_smem(bwd_dq_kernel<R, false>, DqCfg<false>::kSmemBytes) ||
+           set_smem(bwd_dkdv_kernel<R, true>, KvCfg::kSmemBytes) ||
+           set_smem(bwd_dkdv_kernel<R, false>, KvCfg::kSmemBytes);
 }
 
 // Rotated dims the kernels are compiled for (the row is held in registers).
@@ -72,7 +83,8 @@ int device_setup(int *num_sms)
                    set_smem(gswa::full::full_fwd_kernel<0>, gswa::full::kSmemBytes) ||
                    set_smem(gswa::full::full_fwd_kernel<42>, gswa::full::kSmemBytes) ||
                    set_smem(gswa::full::full_fwd_kernel<64>, gswa::full::kSmemBytes) ||
-                   set_smem(gswa::full::full_fwd_kernel<128>, gswa::full::kSmemBytes)) {
+                   set_smem(gswa::full::full_fwd_kernel<128>, gswa::full::kSmemBytes) ||
+                   set_bwd_smem<0>() || set_bwd_smem<42>() || set_bwd_smem<64>() || set_bwd_smem<128>()) {
             d.status = GSWA_ERR_LAUNCH;
         }
         if (d.status == GSWA_OK && g_encode == nullptr) {
@@ -183,6 +195,179 @@ int launch_qk_prep(const gswa_shape_t *s, int H, const void *x, const void *w, v
     case 64: gswa::prep::qk_prep_kernel<64><<<gr, bl, 0, st>>>(pp); break;
     default: gswa::prep::qk_prep_kernel<128><<<gr, bl, 0, st>>>(pp); break;
     }
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
+// Backward workspace: prepared q~ [B,T,Hq,D] and k~ [B,T,Hkv,D] (bf16),
+// dA [B,T,Hq,D] (gated only; ungated dA is dy), the row records
+// [B,Hkv,Tp,4] float2, and the per-warp dw_q / dw_k partials.
+struct BwdWs {
+    size_t qt, kt, da, ld, pq, pk, total;
+};
+
+BwdWs bwd_ws_layout(const gswa_shape_t *s, bool gated)
+{
+    const size_t BT = (size_t)s->B * s->T;
+    const size_t Tp = ((size_t)s->T + 31) / 32 * 32;
+    const size_t part = align256((size_t)gswa::bwd::kMaxGrid * 4 * 128 * 4);
+    BwdWs w;
+    w.qt = 0;
+    w.kt = w.qt + align256(BT * s->Hq * s->D * 2);
+    w.da = w.kt + align256(BT * s->Hkv * s->D * 2);
+    w.ld = w.da + (gated ? align256(BT * s->Hq * s->D * 2) : 0);
+    w.pq = w.ld + align256((size_t)s->B * s->Hkv * Tp * 4 * 8);
+    w.pk = w.pq + part;
+    w.total = w.pk + part;
+    return w;
+}
+
+struct BwdMaps {
+    CUtensorMap tq, ta, tk, tv;       // dq kernel
+    CUtensorMap tk2, tv2, tq2, ta2;   // dk/dv kernel
+};
+
+template <int R, bool kSwa>
+void launch_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::bwd::Params &pk, unsigned gq,
+                     unsigned gk, cudaStream_t st)
+{
+    using namespace gswa::bwd;
+    bwd_dq_kernel<R, kSwa><<<gq, kThreads, DqCfg<kSwa>::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
+    bwd_dkdv_kernel<R, kSwa><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
+}
+
+template <bool kSwa>
+void dispatch_bwd_main(int R, const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::bwd::Params &pk,
+                       unsigned gq, unsigned gk, cudaStream_t st)
+{
+    switch (R) {
+    case 0: launch_bwd_main<0, kSwa>(m, pq, pk, gq, gk, st); break;
+    case 42: launch_bwd_main<42, kSwa>(m, pq, pk, gq, gk, st); break;
+    case 64: launch_bwd_main<64, kSwa>(m, pq, pk, gq, gk, st); break;
+    default: launch_bwd_main<128, kSwa>(m, pq, pk, gq, gk, st); break;
+    }
+}
+
+// Shared body of gswa_bwd (swa: gated sliding window) and full_attn_bwd.
+int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
+            const void *w_q, const void *w_k, const void *y, const float *lse, const void *dy, void *dq,
+            void *dk, void *dv, void *dg, float *dw_q, float *dw_k, void *workspace, size_t workspace_bytes,
+            cudaStream_t st)
+{
+    int rc = check_common(s);
+    if (rc != GSWA_OK) return rc;
+    if (swa && (s->window < 1 || s->window > 128)) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (!rope_dims_supported(s->rope_dims)) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (!dw_q || !dw_k) return GSWA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(dw_q) & 3u) || (reinterpret_cast<uintptr_t>(dw_k) & 3u))
+        return GSWA_ERR_MISALIGNED;
+    int num_sms = 0;
+    if ((long long)s->B * s->T == 0) {
+        // nothing attends: the weight gradients are zero
+        rc = device_setup(&num_sms);
+        if (rc != GSWA_OK) return rc;
+        if (cudaMemsetAsync(dw_q, 0, 128 * sizeof(float), st) != cudaSuccess ||
+            cudaMemsetAsync(dw_k, 0, 128 * sizeof(float), st) != cudaSuccess)
+            return GSWA_ERR_LAUNCH;
+        return GSWA_OK;
+    }
+    if (!q || !k || !v || !w_q || !w_k || !y || !lse || !dy || !dq || !dk || !dv || (swa && (!g || !dg)))
+        return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(dy) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (swa && (!aligned16(g) || !aligned16(dg))) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return GSWA_ERR_MISALIGNED;
+    const BwdWs L = bwd_ws_layout(s, swa);
+    if (workspace == nullptr || workspace_bytes < L.total) return GSWA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
+    rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+
+    char *ws = static_cast<char *>(workspace);
+    void *qt = ws + L.qt, *kt = ws + L.kt;
+    const void *da = swa ? static_cast<const void *>(ws + L.da) : dy;
+    float2 *ld = reinterpret_cast<float2 *>(ws + L.ld);
+    float *part_q = reinterpret_cast<float *>(ws + L.pq), *part_k = reinterpret_cast<float *>(ws + L.pk);
+    const int Tp = (s->T + 31) / 32 * 32;
+
+    // 1. D, lse records, dA, dg
+    gswa::bwd::PrepParams pp;
+    pp.y = static_cast<const __nv_bfloat16 *>(y);
+    pp.dy = static_cast<const __nv_bfloat16 *>(dy);
+    pp.g = static_cast<const __nv_bfloat16 *>(g);
+    pp.lse = lse;
+    pp.dA = swa ? reinterpret_cast<__nv_bfloat16 *>(ws + L.da) : nullptr;
+    pp.dg = static_cast<__nv_bfloat16 *>(dg);
+    pp.ld = ld;
+    pp.rows = (long long)s->B * Tp * s->Hq;
+    pp.T = s->T;
+    pp.Tp = Tp;
+    pp.Hq = s->Hq;
+    long long pgrid = ((long long)s->B * Tp + 15) / 16;   // a half-warp per token
+    if (pgrid > 16LL * num_sms) pgrid = 16LL * num_sms;
+    gswa::bwd::bwd_prep_kernel<<<(unsigned)pgrid, 256, 0, st>>>(pp);
+    // 2. prepared queries and keys
+    rc = launch_qk_prep(s, s->Hq, q, w_q, qt, 0, st, num_sms);
+    if (rc == GSWA_OK) rc = launch_qk_prep(s, s->Hkv, k, w_k, kt, 0, st, num_sms);
+    if (rc != GSWA_OK) return rc;
+
+    // 3. dq and dk/dv
+    const int kN = swa ? gswa::bwd::DqCfg<true>::kN : gswa::bwd::DqCfg<false>::kN;
+    BwdMaps m;
+    if (encode_bthd(&m.tq, qt, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&m.ta, da, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&m.tk, kt, s->B, s->T, s->Hkv, s->D, 1, kN) ||
+        encode_bthd(&m.tv, v, s->B, s->T, s->Hkv, s->D, 1, kN) ||
+        encode_bthd(&m.tk2, kt, s->B, s->T, s->Hkv, s->D, 1, 128) ||
+        encode_bthd(&m.tv2, v, s->B, s->T, s->Hkv, s->D, 1, 128) ||
+        encode_bthd(&m.tq2, qt, s->B, s->T, s->Hq, s->D, 4, gswa::bwd::KvCfg::kChTok) ||
+        encode_bthd(&m.ta2, da, s->B, s->T, s->Hq, s->D, 4, gswa::bwd::KvCfg::kChTok))
+        return GSWA_ERR_INVALID_ARG;
+
+    gswa::bwd::Params pq;
+    std::memset(&pq, 0, sizeof pq);
+    pq.B = s->B;
+    pq.T = s->T;
+    pq.Tp = Tp;
+    pq.Hq = s->Hq;
+    pq.Hkv = s->Hkv;
+    pq.window = swa ? s->window : 0;
+    pq.eps = s->eps;
+    pq.scale = s->scale;
+    pq.sl2 = s->scale * 1.4426950408889634f;
+    pq.ld = ld;
+    fill_theta(pq.theta, s->rope_dims, s->rope_base);
+    gswa::bwd::Params pk = pq;
+
+    pq.nq = Tp / 32;
+    pq.nkt = (s->T + kN - 1) / kN;
+    pq.units = (long long)s->B * s->Hkv * pq.nq;
+    pq.x = static_cast<const __nv_bfloat16 *>(q);
+    pq.w = static_cast<const __nv_bfloat16 *>(w_q);
+    pq.dx = static_cast<__nv_bfloat16 *>(dq);
+    pq.dw_part = part_q;
+
+    pk.nq = pq.nq;
+    pk.nkt = (s->T + 127) / 128;
+    pk.units = (long long)s->B * s->Hkv * pk.nkt;
+    pk.x = static_cast<const __nv_bfloat16 *>(k);
+    pk.w = static_cast<const __nv_bfloat16 *>(w_k);
+    pk.dx = static_cast<__nv_bfloat16 *>(dk);
+    pk.dv = static_cast<__nv_bfloat16 *>(dv);
+    pk.dw_part = part_k;
+
+    auto grid_of = [&](long long units) {
+        long long gsz = units < num_sms ? units : num_sms;
+        return (unsigned)(gsz < gswa::bwd::kMaxGrid ? gsz : gswa::bwd::kMaxGrid);
+    };
+    const unsigned gq = grid_of(pq.units), gk = grid_of(pk.units);
+    if (swa)
+        dispatch_bwd_main<true>(s->rope_dims, m, pq, pk, gq, gk, st);
+    else
+        dispatch_bwd_main<false>(s->rope_dims, m, pq, pk, gq, gk, st);
+    // 4. weight gradients, summed in a fixed order
+    const unsigned rt = gswa::bwd::kD * gswa::bwd::kReduceSlices;
+    gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_q, (int)gq * 4, dw_q);
+    gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_k, (int)gk * 4, dw_k);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
@@ -324,10 +509,8 @@ int gswa_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
              void *dq, void *dk, void *dv, void *dg, float *dw_q, float *dw_k, void *workspace,
              size_t workspace_bytes, void *stream)
 {
-    (void)s; (void)q; (void)k; (void)v; (void)g; (void)w_q; (void)w_k; (void)y; (void)lse;
-    (void)dy; (void)dq; (void)dk; (void)dv; (void)dg; (void)dw_q; (void)dw_k; (void)workspace;
-    (void)workspace_bytes; (void)stream;
-    return GSWA_ERR_UNIMPLEMENTED;
+    return run_bwd(true, s, q, k, v, g, w_q, w_k, y, lse, dy, dq, dk, dv, dg, dw_q, dw_k, workspace,
+                   workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int full_attn_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
@@ -335,10 +518,8 @@ int full_attn_bwd(const gswa_shape_t *s, const void *q, const void *k, const voi
                   const void *dy, void *dq, void *dk, void *dv, float *dw_q, float *dw_k,
                   void *workspace, size_t workspace_bytes, void *stream)
 {
-    (void)s; (void)q; (void)k; (void)v; (void)w_q; (void)w_k; (void)y; (void)lse; (void)dy;
-    (void)dq; (void)dk; (void)dv; (void)dw_q; (void)dw_k; (void)workspace;
-    (void)workspace_bytes; (void)stream;
-    return GSWA_ERR_UNIMPLEMENTED;
+    return run_bwd(false, s, q, k, v, nullptr, w_q, w_k, y, lse, dy, dq, dk, dv, nullptr, dw_q, dw_k, workspace,
+                   workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int gswa_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
@@ -421,6 +602,8 @@ size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
     if (s == nullptr || s->B < 0 || s->T < 0 || s->Hkv <= 0 || s->D <= 0) return 0;
     switch (op) {
     case GSWA_OP_FULL_FWD: return full_fwd_ws(s);
+    case GSWA_OP_GSWA_BWD: return bwd_ws_layout(s, true).total;
+    case GSWA_OP_FULL_BWD: return bwd_ws_layout(s, false).total;
     case GSWA_OP_FULL_DECODE: return s->cache_len > 0 ? full_decode_ws(s) : 0;
     default: return 0;
     }
