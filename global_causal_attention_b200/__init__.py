@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(HERE, "libgswa.so")
 OK = 0
 ERRORS = {
     -1: "INVALID_ARG", -2: "UNSUPPORTED_SHAPE", -3: "MISALIGNED", -4: "WORKSPACE_TOO_SMALL",
-    -5: "LAUNCH", -6: "TIMEOUT", -7: "UNIMPLEMENTED", -8: "NO_DEVICE",
+    -5: "LAUNCH", -6: "TIMEOUT", -7: "UNIMPLEMENTED", -8: "NO_DEVICE", -9: "SCRATCH_LIMIT",
 }
 OP_GSWA_FWD, OP_FULL_FWD, OP_GSWA_BWD, OP_FULL_BWD, OP_GSWA_DECODE, OP_FULL_DECODE = range(6)
 
@@ -63,6 +63,7 @@ def lib():
             "full_attn_bwd": [S] + [P] * 14 + [U, P],
             "gswa_decode": [S] + [P] * 11 + [U, P],
             "full_decode": [S] + [P] * 10 + [U, P],
+            "full_decode_noalloc": [S] + [P] * 10,
             "gswa_qk_prep": [S, I, P, P, P, ctypes.c_int64, P],
         }
         for name, args in sig.items():
@@ -237,6 +238,21 @@ def full_decode(q, k, v, wq, wk, k_cache, v_cache, pos, *, rope_dims=42, rope_ba
     _check(lib().full_decode(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk),
                              _ptr(k_cache), _ptr(v_cache), _ptr(pos), _ptr(y), _ptr(ws), nb,
                              _stream(stream)), "full_decode")
+    return y
+
+
+def full_decode_noalloc(q, k, v, wq, wk, k_cache, v_cache, pos, y, *, rope_dims=42, rope_base=1e4,
+                        eps=1e-6, scale=None, stream=None):
+    """full_decode on the library's fixed device scratch: allocates nothing, so
+    the output y [B, Hq, D] (bf16, cuda) must be passed in.  Calls that can
+    overlap in time share that scratch and must not be issued concurrently."""
+    _dev(q, k, v, wq, wk, k_cache, v_cache, pos, y)
+    B, Hq, D = q.shape
+    s = make_shape(B, 1, Hq, k.shape[1], D, 128, rope_dims, rope_base, eps, scale,
+                   cache_len=k_cache.shape[2])
+    _check(lib().full_decode_noalloc(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk),
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(pos), _ptr(y), _stream(stream)),
+           "full_decode_noalloc")
     return y
 
 

@@ -198,6 +198,40 @@ int launch_qk_prep(const gswa_shape_t *s, int H, const void *x, const void *w, v
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
+// ------------------------------------------------ allocation-free decode
+// The fixed device scratch of full_decode_noalloc: one array per device,
+// placed by the loader with the library's kernels; nothing is allocated at
+// call time.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GSWA_NOALLOC_SCRATCH_BYTES];
+
+struct NoAllocDevice {
+    bool ready = false;
+    int status = GSWA_OK;
+    void *scratch = nullptr;
+};
+NoAllocDevice g_noalloc[kMaxDevices];
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) under the library lock.
+int noalloc_scratch(void **scratch)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GSWA_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    NoAllocDevice &d = g_noalloc[dev];
+    if (!d.ready) {
+        d.ready = true;
+        void *ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr)
+            d.status = GSWA_ERR_LAUNCH;
+        else
+            d.scratch = ptr;
+    }
+    *scratch = d.scratch;
+    return d.status;
+}
+
 // Backward workspace: prepared q~ [B,T,Hq,D] and k~ [B,T,Hkv,D] (bf16),
 // dA [B,T,Hq,D] (gated only; ungated dA is dy), the row records
 // [B,Hkv,Tp,4] float2, and the per-warp dw_q / dw_k partials.
@@ -597,6 +631,48 @@ int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
+int full_decode_noalloc(const gswa_shape_t *s, const void *q, const void *k, const void *v,
+                        const void *w_q, const void *w_k, void *k_cache, void *v_cache,
+                        const int64_t *pos, void *y, void *stream)
+{
+    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->cache_len < 1) return GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
+    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
+        return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->B == 0) return GSWA_OK;
+    if (!q || !k || !v || !w_q || !w_k || !k_cache || !v_cache || !pos || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+        return GSWA_ERR_MISALIGNED;
+    // the same scratch layout full_decode takes from its workspace
+    const size_t q_bytes = align256((size_t)s->B * s->Hq * s->D * 4);
+    if (full_decode_ws(s) > GSWA_NOALLOC_SCRATCH_BYTES) return GSWA_ERR_SCRATCH_LIMIT;
+    int num_sms = 0;
+    int rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    void *scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != GSWA_OK) return rc;
+    gswa::dec::Params p;
+    fill_dec(p, s);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    p.pos = pos;
+    p.y = static_cast<__nv_bfloat16 *>(y);
+    p.qt = static_cast<float *>(scratch);
+    p.part = reinterpret_cast<float *>(static_cast<char *>(scratch) + q_bytes);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
+    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkWarps * 32, 0, st>>>(p);
+    gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
 size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
 {
     if (s == nullptr || s->B < 0 || s->T < 0 || s->Hkv <= 0 || s->D <= 0) return 0;
@@ -645,6 +721,7 @@ const char *gswa_strerror(int code)
     case GSWA_ERR_TIMEOUT: return "a bounded device wait timed out";
     case GSWA_ERR_UNIMPLEMENTED: return "not implemented";
     case GSWA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case GSWA_ERR_SCRATCH_LIMIT: return "shape needs more than the fixed 36 MiB scratch of full_decode_noalloc";
     default: return "unknown error";
     }
 }

@@ -53,6 +53,7 @@ extern "C" {
 #define GSWA_ERR_TIMEOUT (-6)           /* a bounded device wait gave up */
 #define GSWA_ERR_UNIMPLEMENTED (-7)
 #define GSWA_ERR_NO_DEVICE (-8)         /* no sm_100 device current */
+#define GSWA_ERR_SCRATCH_LIMIT (-9)     /* full_decode_noalloc: shape needs more than its fixed scratch */
 
 /* Operation ids for gswa_workspace_bytes(). */
 #define GSWA_OP_GSWA_FWD 0
@@ -148,6 +149,39 @@ int full_decode(const gswa_shape_t *shape, const void *q, const void *k, const v
                 const void *w_q, const void *w_k, void *k_cache, void *v_cache,
                 const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
                 void *stream);
+
+/*
+ * full_decode without a caller-supplied workspace, for callers that may not
+ * allocate device memory at all: an inference loop that runs under a fixed
+ * memory budget or must never stall on an allocator, or plain C code with no
+ * allocator of its own to draw a workspace from.  The ZGCM-1 report has no
+ * counterpart of this entry point; it is a convenience of this library.
+ *
+ * Arguments, layouts, results and the position rules are those of
+ * full_decode.  The scratch it needs (the same gswa_workspace_bytes(
+ * GSWA_OP_FULL_DECODE) bytes) comes from one array of
+ * GSWA_NOALLOC_SCRATCH_BYTES (36 MiB) that the library holds in device
+ * memory, one per device, set aside when the library's kernels are loaded on
+ * that device.  Nothing in that scratch needs to start at zero: every byte a
+ * call reads was written earlier in the same call.
+ *
+ * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ * - The first call on a device does a one-time set-up (it looks up the
+ *   scratch's device address with that device current); make that first call
+ *   before any stream capture begins.
+ * - Shapes that need more than GSWA_NOALLOC_SCRATCH_BYTES are rejected with
+ *   GSWA_ERR_SCRATCH_LIMIT before anything runs.  36 MiB covers, for
+ *   example, 32 sequences of 8 KV heads over a 262,144-token cache
+ *   (33.5 MiB).
+ * - All calls on one device share the one scratch: two calls whose work can
+ *   overlap in time (on different streams, or from different host threads
+ *   without ordering between them) race on it and give wrong results.  Issue
+ *   them on one stream, or order them with events.
+ */
+#define GSWA_NOALLOC_SCRATCH_BYTES ((size_t)36 << 20)
+int full_decode_noalloc(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
+                        const void *w_q, const void *w_k, void *k_cache, void *v_cache,
+                        const int64_t *pos, void *y, void *stream);
 
 /*
  * QK-RMSNorm + partial RoPE of a head tensor on its own (§2.1 Figure 3: the
