@@ -39,12 +39,24 @@ from workloads import WORKLOADS
 METRIC = "gated-SWA/full attn tokens/s (prefill+bwd, decode) and % of roofline, 1 B200"
 UNIT = "tokens/s"
 
-# Hot-path kernels each workload's step runs, in order.
-STEP_OPS = {
-    "train_4k": ["gswa_fwd"],
-    "prefill_64k": ["gswa_fwd"],
-    "prefill_256k": ["gswa_fwd"],
-}
+# What one step of each workload runs (one bench line per workload).
+#   train_4k      one attention layer at training shape, both kinds on the same
+#                 tensors: gated-SWA forward + backward, full causal forward + backward
+#   prefill_64k / prefill_256k   the 32-layer attention stack, forward:
+#                 27 gated-SWA layers + 5 full causal layers (1-based 6, 12, 18, 24, 30)
+#   decode_256k   one decode step of 32 sequences through the 32-layer stack
+#                 (27 ring-cache SWA layers, 5 linear-cache global layers)
+WORKLOAD_NAMES = ["train_4k", "prefill_64k", "prefill_256k", "decode_256k"]
+LAYERS = workloads.N_LAYERS
+
+# Kernel launches of one call of each entry point.
+LAUNCHES = {"gswa_fwd": 1, "gswa_bwd": 7, "full_attn_fwd": 2, "full_attn_bwd": 7, "gswa_decode": 1,
+            "full_decode": 3}
+
+# DRAM bytes (read + write) of one call, from an ncu capture of the same
+# launches (dram__bytes_read.sum + dram__bytes_write.sum summed over the
+# call's kernels); None until captured for the current kernels.
+TRAFFIC = {}
 
 
 def peaks():
@@ -53,14 +65,8 @@ def peaks():
         with open(path) as f:
             p = json.load(f)
         return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
-                    bf16_tflops_sustained=p.get("bf16_tflops_sustained"), source="measured")
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained") or p["bf16_tflops"], source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
-
-
-def swa_fwd_bytes(s) -> int:
-    """Compulsory HBM bytes of one gated-SWA forward: read q, k, v, g; write y, lse."""
-    tok = s.B * s.T
-    return tok * (s.Hq * s.D * 2 * 3 + s.Hkv * s.D * 2 * 2 + s.Hq * 4)
 
 
 def swa_pairs(T: int, W: int) -> int:
@@ -70,9 +76,31 @@ def swa_pairs(T: int, W: int) -> int:
     return W * (W + 1) // 2 + (T - W) * W
 
 
-def swa_fwd_flops(s) -> int:
-    """Algorithmic FLOPs of the two contractions over the unmasked pairs."""
-    return 4 * s.B * s.Hq * s.D * swa_pairs(s.T, s.window)
+def causal_pairs(T: int) -> int:
+    return T * (T + 1) // 2
+
+
+def algorithmic_work(op, s, pos=None):
+    """(bound, amount, unit) of one call: compulsory HBM bytes for the
+    bandwidth-bound calls, useful tensor FLOPs (visible pairs only) for the
+    full causal ones.  Forward: 2 contractions (QK^T, PV) = 4 D FLOPs per
+    pair; backward: 4 (dV, dP, dQ, dK) = 8 D, recomputation not counted."""
+    tok, e = s.B * s.T, 2
+    qb, kb = s.Hq * s.D * e, s.Hkv * s.D * e       # bytes per token of a q-like / k-like tensor
+    if op == "gswa_fwd":      # read q, k, v, g; write y, lse
+        return "hbm", tok * (3 * qb + 2 * kb + s.Hq * 4), "GB/s"
+    if op == "gswa_bwd":      # read q, k, v, g, y, dy, lse; write dq, dk, dv, dg
+        return "hbm", tok * (4 * qb + 2 * kb + s.Hq * 4 + 2 * qb + 2 * kb), "GB/s"
+    if op == "full_attn_fwd":
+        return "tensor", 4 * s.D * s.B * s.Hq * causal_pairs(s.T), "TFLOP/s"
+    if op == "full_attn_bwd":
+        return "tensor", 8 * s.D * s.B * s.Hq * causal_pairs(s.T), "TFLOP/s"
+    if op == "gswa_decode":   # ring K/V of the visible slots + new q, k, v, g, y
+        vis = min(pos + 1, s.window)
+        return "hbm", s.B * (2 * s.Hkv * vis * s.D * e + 3 * s.Hq * s.D * e + 2 * s.Hkv * s.D * e), "GB/s"
+    if op == "full_decode":   # K/V rows 0..pos + new q, k, v, y
+        return "hbm", s.B * (2 * s.Hkv * (pos + 1) * s.D * e + 2 * s.Hq * s.D * e + 2 * s.Hkv * s.D * e), "GB/s"
+    raise ValueError(op)
 
 
 class ClockSampler:
@@ -157,38 +185,155 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
-def make_step(ops, s, x, dev):
-    """Device buffers + a callable running one step; returns (step, outputs, n_launches)."""
+# --------------------------------------------------------------------- workloads
+class Step:
+    """One step of a workload: `calls` is the ordered list of (entry point,
+    callable); `h2d` / `d2h` map device tensors to pinned host copies for the
+    end-to-end variant."""
+
+    def __init__(self, name, s, tokens, calls, h2d, d2h, pos=None):
+        self.name, self.s, self.tokens, self.calls = name, s, tokens, calls
+        self.h2d, self.d2h, self.pos = h2d, d2h, pos
+
+    def ops(self):
+        seen = []
+        for op, _ in self.calls:
+            if op not in seen:
+                seen.append(op)
+        return seen
+
+    def launches(self):
+        return sum(LAUNCHES[op] for op, _ in self.calls)
+
+
+def _ws(gca, op, shape, dev):
+    n = gca.workspace_bytes(op, shape)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+
+
+def build_train(s, dev, seed):
+    """One layer at training shape: gated-SWA fwd+bwd and full causal fwd+bwd on the same tensors."""
     import global_causal_attention_b200 as gca
-    y = torch.empty_like(x["q"])
-    lse = torch.empty((s.B, s.Hq, s.T), dtype=torch.float32, device=dev)
+    x = workloads.attention_inputs(s, seed, device=dev, with_grad=True)
+    kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    sh_swa = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, s.window, **kw)
+    sh_full = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, 0, **kw)
+    e = lambda t: torch.empty_like(t)
+    f32 = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)
+    y_s, y_f = e(x["q"]), e(x["q"])
+    lse_s, lse_f = f32(s.B, s.Hq, s.T), f32(s.B, s.Hq, s.T)
+    g_s = (e(x["q"]), e(x["k"]), e(x["k"]), e(x["q"]), f32(s.D), f32(s.D))
+    g_f = (e(x["q"]), e(x["k"]), e(x["k"]), f32(s.D), f32(s.D))
+    ws_sb = _ws(gca, gca.OP_GSWA_BWD, sh_swa, dev)
+    ws_ff = _ws(gca, gca.OP_FULL_FWD, sh_full, dev)
+    ws_fb = _ws(gca, gca.OP_FULL_BWD, sh_full, dev)
+    q, k, v, g, wq, wk, dy = (x[n] for n in ("q", "k", "v", "g", "wq", "wk", "dy"))
+    calls = [
+        ("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse_s, **kw)),
+        ("gswa_bwd", lambda: gca.gswa_bwd(q, k, v, g, wq, wk, y_s, lse_s, dy, window=s.window, workspace=ws_sb,
+                                          out=g_s, **kw)),
+        ("full_attn_fwd", lambda: gca.full_attn_fwd(q, k, v, wq, wk, y=y_f, lse=lse_f, workspace=ws_ff, **kw)),
+        ("full_attn_bwd", lambda: gca.full_attn_bwd(q, k, v, wq, wk, y_f, lse_f, dy, workspace=ws_fb, out=g_f,
+                                                    **kw)),
+    ]
+    outs = [y_s, y_f, *g_s, *g_f]
+    return Step("train_4k", s, s.B * s.T, calls, x, outs)
 
-    def step():
-        for op in ops:
-            if op == "gswa_fwd":
-                gca.gswa_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
-                             rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale,
-                             y=y, lse=lse)
-            else:
-                raise ValueError(op)
 
-    return step, {"y": y, "lse": lse}, len(ops)
+def build_prefill(name, s, dev, seed):
+    """The 32-layer attention stack, forward, every layer on the same tensors."""
+    import global_causal_attention_b200 as gca
+    x = workloads.attention_inputs(s, seed, device=dev)
+    kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    sh_full = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, 0, **kw)
+    y_s, y_f = torch.empty_like(x["q"]), torch.empty_like(x["q"])
+    lse = torch.empty(s.B, s.Hq, s.T, dtype=torch.float32, device=dev)
+    ws_ff = _ws(gca, gca.OP_FULL_FWD, sh_full, dev)
+    q, k, v, g, wq, wk = (x[n] for n in ("q", "k", "v", "g", "wq", "wk"))
+    calls = []
+    for layer in range(1, LAYERS + 1):
+        if workloads.layer_is_global(layer):
+            calls.append(("full_attn_fwd", lambda: gca.full_attn_fwd(q, k, v, wq, wk, y=y_f, lse=lse,
+                                                                     workspace=ws_ff, **kw)))
+        else:
+            calls.append(("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse,
+                                                           **kw)))
+    return Step(name, s, s.B * s.T, calls, x, [y_s])
 
 
-def time_steps(step, K, W, stream, dist_on, sampler=None):
+def build_decode(dev, seed):
+    """One decode step of 32 sequences through the 32-layer stack.  The five
+    global layers read one 262,144-token linear cache (34 GB of K/V; five
+    distinct caches would not fit in HBM, and a cache this size streams from
+    HBM either way); every SWA layer has its own 128-slot ring."""
+    import global_causal_attention_b200 as gca
+    d = workloads.DECODE_256K
+    B, Hq, Hkv, D, W, Tmax = d["B"], d["Hq"], d["Hkv"], d["D"], d["window"], d["Tmax"]
+    s = workloads.Shape(B=B, T=1, Hq=Hq, Hkv=Hkv, window=W, rope_base=d["rope_base"])
+    kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    kc = workloads.fill_randn_bf16_(torch.empty(B, Hkv, Tmax, D, **bf), seed * 100 + 1)
+    vc = workloads.fill_randn_bf16_(torch.empty(B, Hkv, Tmax, D, **bf), seed * 100 + 2)
+    pos = torch.full((B,), d["pos"], dtype=torch.int64, device=dev)
+    wq = torch.ones(D, **bf)
+    wk = torch.ones(D, **bf)
+    ws_fd = _ws(gca, gca.OP_FULL_DECODE, gca.make_shape(B, 1, Hq, Hkv, D, W, cache_len=Tmax, **kw), dev)
+    calls, h2d, y = [], {"pos": pos}, None
+    for layer in range(1, LAYERS + 1):
+        li = workloads.decode_inputs(B, Hq, Hkv, D, 1, seed=seed * 64 + layer, device=dev)
+        q, k, v, g = li["q"], li["k"], li["v"], li["g"]
+        for n in ("q", "k", "v", "g"):
+            h2d[f"{n}{layer}"] = li[n]
+        y = torch.empty_like(q)
+        if workloads.layer_is_global(layer):
+            calls.append(("full_decode", lambda q=q, k=k, v=v, y=y: gca.full_decode(
+                q, k, v, wq, wk, kc, vc, pos, y=y, workspace=ws_fd, **kw)))
+        else:
+            kr = workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 10 + layer)
+            vr = workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 50 + layer)
+            calls.append(("gswa_decode", lambda q=q, k=k, v=v, g=g, kr=kr, vr=vr, y=y: gca.gswa_decode(
+                q, k, v, g, wq, wk, kr, vr, pos, y=y, **kw)))
+    return Step("decode_256k", s, B, calls, h2d, [y], pos=d["pos"])
+
+
+def build(name, dev, seed):
+    if name == "train_4k":
+        return build_train(WORKLOADS["train_4k"], dev, seed)
+    if name in ("prefill_64k", "prefill_256k"):
+        return build_prefill(name, WORKLOADS[name], dev, seed)
+    if name == "decode_256k":
+        return build_decode(dev, seed)
+    raise ValueError(name)
+
+
+# ---------------------------------------------------------------------- timing
+def time_steps(step, K, W, stream, dist_on, sampler=None, per_op=False):
+    """Device time of K steps after W warm-up steps (ms, max over ranks) and,
+    with per_op, the summed device time of each entry point over the K steps,
+    from CUDA events recorded around every call on the launching stream."""
+    def run_one(evs=None):
+        for i, (op, fn) in enumerate(step.calls):
+            if evs is not None:
+                evs[2 * i].record(stream)
+            fn()
+            if evs is not None:
+                evs[2 * i + 1].record(stream)
+
     for _ in range(W):
-        step()
+        run_one()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(step.calls))] for _ in range(K)] \
+        if per_op else [None] * K
     if sampler is not None:
         sampler.__enter__()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(K):
-        step()
+    for kk in range(K):
+        run_one(evsets[kk])
     e1.record(stream)
     torch.cuda.synchronize()
     if sampler is not None:
@@ -196,105 +341,207 @@ def time_steps(step, K, W, stream, dist_on, sampler=None):
     if dist_on:
         torch.distributed.barrier()
     ms = e0.elapsed_time(e1)
+    op_ms = {}
+    if per_op:
+        for evs in evsets:
+            for i, (op, _) in enumerate(step.calls):
+                op_ms[op] = op_ms.get(op, 0.0) + evs[2 * i].elapsed_time(evs[2 * i + 1])
     if dist_on:
         t = torch.tensor([ms], device="cuda")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    return ms
+    return ms, op_ms
 
 
-def launch_ms(fn, reps, stream):
-    """Average duration of one launch of `fn`, CUDA events on its stream."""
-    fn()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        fn()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
+def op_table(step, op_ms, K, pk):
+    """Per entry point: calls per step, ms per call, achieved rate against its bound."""
+    table = {}
+    for op in step.ops():
+        n = sum(1 for o, _ in step.calls if o == op)
+        per_call = op_ms[op] / (K * n)
+        bound, amount, unit = algorithmic_work(op, step.s, step.pos)
+        if bound == "hbm":
+            achieved, peak = amount / (per_call / 1e3) / 1e9, pk["hbm_gbs"]
+        else:
+            achieved, peak = amount / (per_call / 1e3) / 1e12, pk["bf16_tflops_sustained"]
+        table[op] = {"calls_per_step": n, "ms_per_call": per_call, "bound": bound, "achieved": achieved,
+                     "unit": unit, "peak": peak, "frac": achieved / peak,
+                     "algorithmic_per_call": amount, "launches_per_call": LAUNCHES[op]}
+    return table
 
 
-def cpu_baseline(s, target_s=15.0):
-    """The float64 oracle on a bounded sample of the workload's query rows."""
+# ---------------------------------------------------------------- the oracle
+def _oracle_cores():
     import oracle
-    from workloads import attention_inputs, sample_rows
-    x = attention_inputs(s, 0)
-    nrows = 8
-    spent = 0.0
-    while True:
-        rows = sample_rows(s.T, nrows, seed=3).numpy()
+    return oracle.num_threads()
+
+
+_ORACLE_INPUTS = {}
+
+
+def _memo(key, make):
+    """Oracle inputs are generated once per process (a 262,144-token cache takes seconds)."""
+    if key not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS[key] = make()
+    return _ORACLE_INPUTS[key]
+
+
+def oracle_sample(name, budget_s):
+    """Run the float64 oracle on a bounded sample of one step of `name` and
+    extrapolate to the whole step.  Returns (measured s, extrapolated s for one
+    full step, threads used, description)."""
+    import oracle
+    cores = _oracle_cores()
+    if name == "train_4k":
+        s = WORKLOADS["train_4k"]
+        # one sequence's causal prefix of T' tokens over G' KV groups: the outputs of a
+        # prefix depend on the prefix only, so this is an exact slice of the step
+        G = max(1, min(s.Hkv, cores)) if budget_s >= 10 else 1
+        Tp = s.T if budget_s >= 10 else max(128, min(s.T, int(math.sqrt(budget_s / 1.1e-6)) // 128 * 128))
+        sg = s.replace(B=1, T=Tp, Hq=4 * G, Hkv=G)
+        x = _memo(("train", Tp, G), lambda: workloads.attention_inputs(sg, 0, with_grad=True))
+        kw = oracle.shape_kwargs(sg)
         t0 = time.perf_counter()
-        oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
-                        gated=True, rows=rows, **oracle.shape_kwargs(s))
-        spent = time.perf_counter() - t0
-        if spent * 2 > target_s or nrows >= s.T:
-            break
-        nrows = min(s.T, nrows * max(2, int(target_s / max(spent, 1e-3) / 2)))
-    tokens = s.B * len(rows)
-    return {"value": tokens / spent, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"gated-SWA forward of {len(rows)} seeded query positions x {s.B} sequences "
-                      f"x all {s.Hq} heads of {s.B}x{s.T} (keys prepared for every position), "
-                      f"float64, {spent:.1f} s"}
+        oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window, gated=True, **kw)
+        oracle.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], x["dy"], window=s.window, gated=True,
+                        **kw)
+        t1 = time.perf_counter()
+        oracle.attn_fwd(x["q"], x["k"], x["v"], None, x["wq"], x["wk"], window=0, gated=False, **kw)
+        oracle.attn_bwd(x["q"], x["k"], x["v"], None, x["wq"], x["wk"], x["dy"], window=0, gated=False, **kw)
+        t2 = time.perf_counter()
+        groups = s.B * s.Hkv / G
+        full = (t1 - t0) * groups * swa_pairs(s.T, s.window) / swa_pairs(Tp, s.window) + \
+               (t2 - t1) * groups * causal_pairs(s.T) / causal_pairs(Tp)
+        desc = (f"gated-SWA fwd+bwd and full causal fwd+bwd of the first {Tp} tokens of 1 sequence x {G} of "
+                f"{s.Hkv} KV groups ({4 * G} query heads), float64; extrapolated to {s.B}x{s.T}x{s.Hq} heads "
+                f"by the exact visible-pair counts of each part")
+        return t2 - t0, full, min(G, cores), desc
+    if name in ("prefill_64k", "prefill_256k"):
+        s = WORKLOADS[name]
+        # about 0.1 s of oracle work per sampled row at 64K (rows cost in proportion to position)
+        nrows = max(2, min(256, int(budget_s / (0.12 * s.T / 65536))))
+        rows = workloads.sample_rows(s.T, nrows, seed=3).numpy()
+        G = min(s.Hkv, cores)
+        sg = s.replace(B=1, Hq=4 * G, Hkv=G)
+        x = _memo((name, G), lambda: workloads.attention_inputs(sg, 0))
+        kw = oracle.shape_kwargs(sg)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window, gated=True,
+                        rows=rows, **kw)
+        t1 = time.perf_counter()
+        oracle.attn_fwd(x["q"], x["k"], x["v"], None, x["wq"], x["wk"], window=0, gated=False, rows=rows, **kw)
+        t2 = time.perf_counter()
+        groups = s.B * s.Hkv / G
+        n_swa = sum(1 for l in range(1, LAYERS + 1) if not workloads.layer_is_global(l))
+        n_full = LAYERS - n_swa
+        ps = sum(min(int(i) + 1, s.window) for i in rows)
+        pf = sum(int(i) + 1 for i in rows)
+        full = n_swa * (t1 - t0) * groups * swa_pairs(s.T, s.window) / ps + \
+               n_full * (t2 - t1) * groups * causal_pairs(s.T) / pf
+        desc = (f"gated-SWA and full causal forward of {len(rows)} seeded query positions of 1 sequence x {G} KV "
+                f"groups ({4 * G} query heads) at T={s.T}, float64; extrapolated to the {n_swa}+{n_full}-layer "
+                f"stack by the exact visible-pair counts (the per-call key preparation is not scaled)")
+        return t2 - t0, full, min(G, cores), desc
+    if name == "decode_256k":
+        d = workloads.DECODE_256K
+        s = workloads.Shape(B=1, T=1, Hq=d["Hq"], Hkv=d["Hkv"], window=d["window"], rope_base=d["rope_base"])
+        kw = oracle.shape_kwargs(s)
+        xs = _memo("ring", lambda: workloads.decode_inputs(1, d["Hq"], d["Hkv"], d["D"], d["window"], seed=0))
+        pos = [d["pos"]]
+        xf = _memo("linear", lambda: workloads.decode_inputs(1, d["Hq"], d["Hkv"], d["D"], d["Tmax"], seed=0))
+        reps = max(1, min(d["B"], int(budget_s / 0.4)))   # about 0.4 s per repetition
+        t_swa = t_full = 0.0
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            oracle.decode(xs["q"], xs["k"], xs["v"], xs["g"], xs["wq"], xs["wk"], xs["k_cache"], xs["v_cache"],
+                          pos, window=d["window"], gated=True, **kw)
+            t1 = time.perf_counter()
+            oracle.decode(xf["q"], xf["k"], xf["v"], None, xf["wq"], xf["wk"], xf["k_cache"], xf["v_cache"],
+                          pos, window=0, gated=False, **kw)
+            t2 = time.perf_counter()
+            t_swa += t1 - t0
+            t_full += t2 - t1
+        n_full = sum(1 for l in range(1, LAYERS + 1) if workloads.layer_is_global(l))
+        full = d["B"] * ((LAYERS - n_full) * t_swa + n_full * t_full) / reps
+        desc = (f"{reps} x (one SWA-layer ring decode and one global-layer 262,144-token-cache decode) of one "
+                f"sequence, float64; extrapolated to {d['B']} sequences and the 27+5-layer stack")
+        return t_swa + t_full, full, min(d["Hkv"], cores), desc
+    raise ValueError(name)
+
+
+def cpu_baseline(name, tokens):
+    measured, full, cores, desc = oracle_sample(name, budget_s=15.0)
+    return {"value": tokens / full, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{desc}; {measured:.1f} s measured"}
 
 
 def run_reference(args):
-    """--impl reference: the oracle, timed on the host cores, same metric/config."""
+    """--impl reference: the oracle, timed on the host cores, same metric and config."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    s = WORKLOADS[args.workload]
-    import oracle
-    from workloads import attention_inputs, sample_rows
-    x = attention_inputs(s, 0)
-    rows = sample_rows(s.T, 16, seed=3).numpy()
-    kw = oracle.shape_kwargs(s)
-
-    def step():
-        oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window,
-                        gated=True, rows=rows, **kw)
-
+    budget = 120.0 / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
+        oracle_sample(args.workload, budget)
+    measured = extrap = 0.0
+    desc, cores = "", 1
     for _ in range(args.steps):
-        step()
-    dt = time.perf_counter() - t0
-    tokens = s.B * len(rows) * args.steps
-    value = tokens / dt
-    sample = (f"gated-SWA forward of {len(rows)} seeded query positions x {s.B} sequences x all "
-              f"{s.Hq} heads of {s.B}x{s.T} per step, float64")
+        m, e, cores, desc = oracle_sample(args.workload, budget)
+        measured += m
+        extrap += e
+    tokens = tokens_per_step(args.workload)
+    value = tokens * args.steps / extrap
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": workload_config(s, args.workload, STEP_OPS[args.workload], args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": sample},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": extrap * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.workload, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}; {measured:.1f} s measured over {args.steps} steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def workload_config(s, name, ops, n):
-    return {"workload": f"{name}: " + " + ".join(ops) + f" (B{s.B} T{s.T} {s.Hq}q/{s.Hkv}kv "
-                        f"D{s.D} W{s.window} rope {s.rope_dims}/{s.D} base {s.rope_base:g})",
+def tokens_per_step(name):
+    if name == "decode_256k":
+        return workloads.DECODE_256K["B"]
+    s = WORKLOADS[name]
+    return s.B * s.T
+
+
+def workload_config(name, n):
+    if name == "decode_256k":
+        d = workloads.DECODE_256K
+        return {"workload": f"decode_256k: one decode step of {d['B']} sequences at position {d['pos']} through "
+                            f"the 32-layer stack (27 gswa_decode on 128-slot rings + 5 full_decode on a "
+                            f"{d['Tmax']}-token linear cache), {d['Hq']}q/{d['Hkv']}kv D{d['D']}, base "
+                            f"{d['rope_base']:g}",
+                "global_batch": d["B"] * n, "seq_len": d["Tmax"], "parallelism": f"replicas x{n} (weak)",
+                "l2": "caches larger than L2 (no flush needed)"}
+    s = WORKLOADS[name]
+    what = ("gswa_fwd + gswa_bwd + full_attn_fwd + full_attn_bwd on the same tensors" if name == "train_4k"
+            else "32-layer stack forward: 27 gswa_fwd + 5 full_attn_fwd (layers 6, 12, 18, 24, 30)")
+    return {"workload": f"{name}: {what} (B{s.B} T{s.T} {s.Hq}q/{s.Hkv}kv D{s.D} W{s.window} "
+                        f"rope {s.rope_dims}/{s.D} base {s.rope_base:g})",
             "global_batch": s.B * n, "seq_len": s.T, "parallelism": f"replicas x{n} (weak)",
             "l2": "inputs larger than L2 (no flush needed)"}
+
+
+DEFAULT_STEPS = {"train_4k": 100, "prefill_64k": 5, "prefill_256k": 2, "decode_256k": 30}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="train_4k", choices=sorted(STEP_OPS))
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="train_4k", choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
     if args.impl == "reference":
         run_reference(args)
         return
@@ -312,61 +559,62 @@ def main():
 
     import global_causal_attention_b200 as gca
     gca.lib()
-    s = WORKLOADS[args.workload]
-    ops = STEP_OPS[args.workload]
-    x = workloads.attention_inputs(s, seed=rank, device=dev)
+    step = build(args.workload, dev, seed=rank)
     stream = torch.cuda.current_stream(dev)
-    step, outs, launches_per_step = make_step(ops, s, x, dev)
 
     clk = ClockSampler(torch.cuda.current_device())
-    ms = time_steps(step, args.steps, args.warmup, stream, dist_on, sampler=clk)
+    ms, op_ms = time_steps(step, args.steps, args.warmup, stream, dist_on, sampler=clk, per_op=True)
     clocks = clk.summary()
     if gca.gswa_check_status() != 0:
-        raise RuntimeError("device status reports a timed-out wait")
-    tokens_per_step = s.B * s.T * world
-    value = tokens_per_step * args.steps / (ms / 1e3)
+        raise RuntimeError("device status reports a timed-out wait or a bad position")
+    tokens = step.tokens * world
+    value = tokens * args.steps / (ms / 1e3)
 
-    # Roofline of the dominant kernel (the gated-SWA forward: HBM-bound).
     pk = peaks()
-    fwd_ms = launch_ms(step, 10, stream)
-    fwd_bytes = swa_fwd_bytes(s)
-    achieved = fwd_bytes / (fwd_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "gswa_fwd", "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "algorithmic_bytes_per_launch": fwd_bytes, "launch_ms": fwd_ms,
-                "peak_source": pk["source"], "tensor_tflops": swa_fwd_flops(s) / (fwd_ms / 1e3) / 1e12}
+    ops = op_table(step, op_ms, args.steps, pk)
+    dom = max(ops, key=lambda o: ops[o]["ms_per_call"] * ops[o]["calls_per_step"])
+    d = ops[dom]
+    roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
+                "frac": d["frac"], "traffic": TRAFFIC.get((args.workload, dom)), "kernel": dom,
+                "launches": d["launches_per_call"], "ms_per_launch": d["ms_per_call"],
+                "algorithmic_per_launch": d["algorithmic_per_call"],
+                "peak_source": pk["source"] + (" sustained" if d["bound"] == "tensor" else "")}
 
-    # End to end through the public API: pinned host inputs -> device, step,
-    # output back to the host, every step.
-    host = {n: t.to("cpu").pin_memory() for n, t in x.items()}
-    y_host = torch.empty(outs["y"].shape, dtype=outs["y"].dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = y_host.numel() * y_host.element_size()
+    # End to end through the public API: the step's inputs copied from pinned
+    # host memory to the device and its outputs back, every step.
+    host_in = {n: t.to("cpu").pin_memory() for n, t in step.h2d.items()}
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.d2h]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    calls = step.calls
 
-    def e2e_step():
-        for n, t in host.items():
-            x[n].copy_(t, non_blocking=True)
-        step()
-        y_host.copy_(outs["y"], non_blocking=True)
+    def e2e_calls():
+        for n, t in host_in.items():
+            step.h2d[n].copy_(t, non_blocking=True)
+        for _, fn in calls:
+            fn()
+        for h, t in zip(host_out, step.d2h):
+            h.copy_(t, non_blocking=True)
 
-    e2e_steps = max(2, min(args.steps, 5))
-    e2e_ms = time_steps(e2e_step, e2e_steps, 1, stream, dist_on)
-    e2e_value = tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    e2e_step = Step(step.name, step.s, step.tokens, [("e2e", e2e_calls)], {}, [])
+    e2e_k = max(2, min(args.steps, 5))
+    e2e_ms, _ = time_steps(e2e_step, e2e_k, 1, stream, dist_on)
+    e2e_value = tokens * e2e_k / (e2e_ms / 1e3)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(s)
+        cpu = cpu_baseline(args.workload, step.tokens)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(s, args.workload, ops, world),
+            "config": workload_config(args.workload, world),
             "roofline": roofline,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
+            "ops": ops,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": step.launches() * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

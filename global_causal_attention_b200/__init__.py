@@ -170,13 +170,14 @@ def _bwd_outputs(q, k, gated):
 
 
 def gswa_bwd(q, k, v, g, wq, wk, y, lse, dy, *, window=128, rope_dims=42, rope_base=1e4, eps=1e-6,
-             scale=None, workspace=None, stream=None):
+             scale=None, workspace=None, out=None, stream=None):
     """Backward of gswa_fwd given its y and lse and the upstream dy [B,T,Hq,D].
-    Returns (dq, dk, dv, dg) bf16 and (dw_q, dw_k) f32."""
-    _dev(q, k, v, g, wq, wk, y, lse, dy)
+    Returns (dq, dk, dv, dg) bf16 and (dw_q, dw_k) f32, written into `out`
+    (a tuple of those six tensors) when given."""
+    _dev(q, k, v, g, wq, wk, y, lse, dy, *(out or ()))
     B, T, Hq, D = q.shape
     s = make_shape(B, T, Hq, k.shape[2], D, window, rope_dims, rope_base, eps, scale)
-    dq, dk, dv, dg, dwq, dwk = _bwd_outputs(q, k, True)
+    dq, dk, dv, dg, dwq, dwk = out if out is not None else _bwd_outputs(q, k, True)
     ws, nb = _workspace(OP_GSWA_BWD, s, workspace, q.device)
     _check(lib().gswa_bwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk), _ptr(y),
                           _ptr(lse), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dwq), _ptr(dwk),
@@ -185,12 +186,16 @@ def gswa_bwd(q, k, v, g, wq, wk, y, lse, dy, *, window=128, rope_dims=42, rope_b
 
 
 def full_attn_bwd(q, k, v, wq, wk, y, lse, dy, *, rope_dims=42, rope_base=1e4, eps=1e-6, scale=None,
-                  workspace=None, stream=None):
-    """Backward of full_attn_fwd.  Returns (dq, dk, dv) bf16 and (dw_q, dw_k) f32."""
-    _dev(q, k, v, wq, wk, y, lse, dy)
+                  workspace=None, out=None, stream=None):
+    """Backward of full_attn_fwd.  Returns (dq, dk, dv) bf16 and (dw_q, dw_k) f32,
+    written into `out` (those five tensors) when given."""
+    _dev(q, k, v, wq, wk, y, lse, dy, *(out or ()))
     B, T, Hq, D = q.shape
     s = make_shape(B, T, Hq, k.shape[2], D, 0, rope_dims, rope_base, eps, scale)
-    dq, dk, dv, _, dwq, dwk = _bwd_outputs(q, k, False)
+    if out is not None:
+        dq, dk, dv, dwq, dwk = out
+    else:
+        dq, dk, dv, _, dwq, dwk = _bwd_outputs(q, k, False)
     ws, nb = _workspace(OP_FULL_BWD, s, workspace, q.device)
     _check(lib().full_attn_bwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(y),
                                _ptr(lse), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dwq), _ptr(dwk),
