@@ -347,10 +347,15 @@ def time_steps(step, K, W, stream, dist_on, sampler=None, per_op=False):
             for i, (op, _) in enumerate(step.calls):
                 op_ms[op] = op_ms.get(op, 0.0) + evs[2 * i].elapsed_time(evs[2 * i + 1])
     if dist_on:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, "cuda")
     return ms, op_ms
+
+
+def max_over_ranks(ms, device):
+    """The slowest rank's time: every rank contributes its own and gets the max."""
+    t = torch.tensor([float(ms)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def op_table(step, op_ms, K, pk):
