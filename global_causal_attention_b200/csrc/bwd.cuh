@@ -521,7 +521,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             ws.init(p);
             wd.init(p);
             int ns = 0, nd = 0;
-            uint64_t t_last = globaltimer();
+            PollWatch watch;
             while (wd.valid) {
                 bool progressed = false;
                 if (ws.valid && ns < nd + kNBuf && mbar_test(bar(C::BQ_FULL), ws.k & 1) &&
@@ -567,15 +567,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     ++nd;
                     progressed = true;
                 }
-                if (progressed) {
-                    t_last = globaltimer();
-                } else {
-                    if (ab.raised()) break;
-                    if (globaltimer() - t_last > kWaitLimitNs) {
-                        ab.raise(kStatusTimeout);
-                        break;
-                    }
-                }
+                if (!watch.tick(progressed, ab)) break;
             }
             mma_commit(bar(C::B_DRAIN));
             drain_wait(bar(C::B_DRAIN), 0);
@@ -662,30 +654,342 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
-// ============================================================ dk/dv kernel
-struct KvCfg {
-    static constexpr int kM = 64;                    // query rows per chunk (16 tokens x 4 heads)
-    static constexpr int kChTok = 16;
+// Row `row` of a swizzled two-half shared-memory tile (halves `hs` bytes
+// apart), 128 bf16, into 64 TMEM columns of this thread's lane from `taddr`
+// (bf16 pairs, the layout of a TMEM A operand).
+__device__ __forceinline__ void smem_row_to_tmem(uint32_t tile, uint32_t hs, int row, uint32_t taddr)
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v = lds128(tile + swa::chunk_off(row, 4 * q + c, hs));
+            w[4 * c] = v.x;
+            w[4 * c + 1] = v.y;
+            w[4 * c + 2] = v.z;
+            w[4 * c + 3] = v.w;
+        }
+        tmem_st16(taddr + 16 * q, w);
+    }
+}
+
+// Store 32 consecutive bf16 (16 packed words) as chunks c0 .. c0 + 3 of row
+// `row` of a single-half swizzled K-major tile (128-byte rows).
+__device__ __forceinline__ void sts_row_chunks(uint32_t tile, int row, int c0, const uint32_t (&w)[16])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        sts128(tile + (uint32_t)row * kHalfRowBytes + ((uint32_t)((c0 + q) ^ (row & 7)) << 4),
+               make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+}
+
+// ====================================================== dq kernel, full causal
+// Query-stationary (M = 128 rows = 4 heads x 32 tokens) over 64-key tiles.
+// The unit's Q~ and dA are copied once into TMEM, so S = Q~K~^T and
+// dP = dA V^T take their A operand from TMEM (two TMEM buffers).  Eight warps
+// (two per TMEM lane quarter, 32 of the 64 key columns each) load S and dP,
+// release the buffer, and write dS as bf16 into shared memory, from where
+// dQ~ += dS K~ reads it.  Warps 4-7 run the epilogue.
+struct DqFullCfg {
+    static constexpr int kN = 64;
     static constexpr int kStages = 4;
-    static constexpr uint32_t kKHalf = 128 * kHalfRowBytes;   // 16 KiB
+    static constexpr uint32_t kQHalf = 128 * kHalfRowBytes;
+    static constexpr uint32_t kQTile = 2 * kQHalf;
+    static constexpr uint32_t kKHalf = kN * kHalfRowBytes;
     static constexpr uint32_t kKTile = 2 * kKHalf;
-    static constexpr uint32_t kCHalf = kM * kHalfRowBytes;    // 8 KiB
-    static constexpr uint32_t kCTile = 2 * kCHalf;
-    static constexpr uint32_t kStageBytes = 2 * kCTile + 1024;   // Q~ chunk, dA chunk, records (512 B)
-    static constexpr uint32_t kOffK = 0;
-    static constexpr uint32_t kOffV = kOffK + kKTile;
-    static constexpr uint32_t kOffCh = kOffV + kKTile;
-    static constexpr uint32_t kOffW = kOffCh + kStages * kStageBytes;
+    static constexpr uint32_t kDSTile = 128 * kHalfRowBytes;   // dS: 128 rows x 64 keys bf16
+    static constexpr uint32_t kOffQ = 0;
+    static constexpr uint32_t kOffA = kOffQ + kQTile;
+    static constexpr uint32_t kOffK = kOffA + kQTile;
+    static constexpr uint32_t kOffV = kOffK + kStages * kKTile;
+    static constexpr uint32_t kOffDS = kOffV + kStages * kKTile;
+    static constexpr uint32_t kOffW = kOffDS + kDSTile;
     static constexpr uint32_t kOffBar = kOffW + 512;
     static constexpr int kNumBars = 24;
     static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
     static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
-    static constexpr uint32_t kColDV = 256, kColDK = 384;
+    // TMEM columns: Q~, dA (A operands), two {S, dP} buffers, dQ~
+    static constexpr uint32_t kColQ = 0, kColA = 64, kColBuf = 128, kBufStride = 128, kColDQ = 384;
+    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    static constexpr int BQ_FULL = 0, BQ_EMPTY = 1, BSTAT = 2, BKV_FULL = 3, BKV_EMPTY = BKV_FULL + kStages,
+                         BS_FULL = BKV_EMPTY + kStages, BS_FREE = BS_FULL + 2, BDS_READY = BS_FREE + 2,
+                         BDS_FREE = BDS_READY + 1, BACC_FULL = BDS_FREE + 1, BACC_FREE = BACC_FULL + 1,
+                         B_DRAIN = BACC_FREE + 1;
+    static_assert(B_DRAIN < kNumBars, "barrier count");
+};
+
+static_assert(DqFullCfg::kN == DqCfg<false>::kN, "full-causal dq units are walked with the 64-key tiling");
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_full_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ Params p)
+{
+    using C = DqFullCfg;
+    constexpr int kN = C::kN, kStages = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    Abort ab{reinterpret_cast<volatile int *>(smem + C::kOffAbort)};
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * (uint32_t)i; };
+    const int nunits = snake_count(p.units);
+
+    if (tid == 0) {
+        *ab.flag = 0;
+        mbar_init(bar(C::BQ_FULL), 1);
+        mbar_init(bar(C::BQ_EMPTY), 8);
+        mbar_init(bar(C::BSTAT), 8);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(bar(C::BKV_FULL + i), 1);
+            mbar_init(bar(C::BKV_EMPTY + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::BS_FULL + i), 1);
+            mbar_init(bar(C::BS_FREE + i), 8);
+        }
+        mbar_init(bar(C::BDS_READY), 8);
+        mbar_init(bar(C::BDS_FREE), 1);
+        mbar_init(bar(C::BACC_FULL), 1);
+        mbar_init(bar(C::BACC_FREE), 4);
+        mbar_init(bar(C::B_DRAIN), 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (tid < 128) reinterpret_cast<float *>(smem + C::kOffW)[tid] = __bfloat162float(p.w[tid]);
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            int g = 0, k = 0;
+            QUnit x;
+            bool ok = true;
+            for (; k < nunits && ok; ++k) {
+                dq_unit_at<false>(p, k, x);
+                ok = mbar_wait(bar(C::BQ_EMPTY), (k & 1) ^ 1u, ab);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(C::BQ_FULL), 2 * C::kQTile);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_4d(sbase + C::kOffQ + h * C::kQHalf, &tm_q, bar(C::BQ_FULL), h * 64, x.kvh * 4,
+                                x.qb * 32, x.b);
+                    tma_load_4d(sbase + C::kOffA + h * C::kQHalf, &tm_a, bar(C::BQ_FULL), h * 64, x.kvh * 4,
+                                x.qb * 32, x.b);
+                }
+                for (int j = 0; j < x.n && ok; ++j, ++g) {
+                    const int st = g % kStages;
+                    ok = mbar_wait(bar(C::BKV_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(bar(C::BKV_FULL + st), 2 * C::kKTile);
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_4d(sbase + C::kOffK + st * C::kKTile + h * C::kKHalf, &tm_k,
+                                    bar(C::BKV_FULL + st), h * 64, x.kvh, j * kN, x.b);
+                        tma_load_4d(sbase + C::kOffV + st * C::kKTile + h * C::kKHalf, &tm_v,
+                                    bar(C::BKV_FULL + st), h * 64, x.kvh, j * kN, x.b);
+                    }
+                }
+            }
+            for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
+                drain_wait(bar(C::BKV_FULL + i % kStages), (i / kStages) & 1);
+            if (k > 0) drain_wait(bar(C::BQ_FULL), (k - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, kN, 0, 0);
+            const uint32_t idesc_dq = idesc_bf16_f32(128, 128, 0, 1);
+            DqWalk<false> ws, wd;
+            ws.init(p);
+            wd.init(p);
+            int ns = 0, nd = 0;
+            PollWatch watch;
+            while (wd.valid) {
+                bool progressed = false;
+                if (ws.valid && ns < nd + 2 && mbar_test(bar(C::BSTAT), ws.k & 1) &&
+                    mbar_test(bar(C::BKV_FULL + ns % kStages), (ns / kStages) & 1) &&
+                    mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
+                    tc_fence_after();
+                    const uint32_t dS = tmem + C::kColBuf + (ns & 1) * C::kBufStride;
+                    const uint32_t ks = sbase + C::kOffK + (ns % kStages) * C::kKTile;
+                    const uint32_t vs = sbase + C::kOffV + (ns % kStages) * C::kKTile;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        mma_ts(dS, tmem + C::kColQ + kk * 8, smem_desc_sw128(ks + ok_, 16, 1024), idesc_s, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
+                        mma_ts(dS + kN, tmem + C::kColA + kk * 8, smem_desc_sw128(vs + ok_, 16, 1024), idesc_s,
+                               kk > 0);
+                    }
+                    mma_commit(bar(C::BS_FULL + (ns & 1)));
+                    ws.next(p);
+                    ++ns;
+                    progressed = true;
+                }
+                if (nd < ns && mbar_test(bar(C::BDS_READY), nd & 1) &&
+                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
+                    tc_fence_after();
+                    const uint32_t ks = sbase + C::kOffK + (nd % kStages) * C::kKTile;
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk)
+                        mma_ss(tmem + C::kColDQ, smem_desc_sw128(sbase + C::kOffDS + kk * 32, 16, 1024),
+                               smem_desc_sw128(ks + kk * 16 * 128, C::kKHalf, 1024), idesc_dq, (wd.j > 0 || kk > 0));
+                    mma_commit(bar(C::BKV_EMPTY + nd % kStages));
+                    mma_commit(bar(C::BDS_FREE));
+                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
+                    wd.next(p);
+                    ++nd;
+                    progressed = true;
+                }
+                if (!watch.tick(progressed, ab)) break;
+            }
+            mma_commit(bar(C::B_DRAIN));
+            drain_wait(bar(C::B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ================================================= Q~/dA into TMEM; dS (8 warps); epilogue (warps 4-7)
+        const int grp = (warp - 4) >> 2;           // key-column half of each tile
+        const int r = 32 * (warp & 3) + lane;      // query row (TMEM lane)
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
+        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
+        bool ok = true;
+        int g = 0;
+        QUnit x;
+        for (int k = 0; k < nunits && ok; ++k) {
+            dq_unit_at<false>(p, k, x);
+            // every MMA reading the previous unit's Q~/dA has completed: this warp
+            // consumed the S/dP of that unit's last tile
+            ok = warp_wait(bar(C::BQ_FULL), k & 1, ab);
+            if (!ok) break;
+            if (grp == 0)
+                smem_row_to_tmem(sbase + C::kOffQ, C::kQHalf, r, tmem + lane_base + C::kColQ);
+            else
+                smem_row_to_tmem(sbase + C::kOffA, C::kQHalf, r, tmem + lane_base + C::kColA);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(C::BSTAT));
+                mbar_arrive(bar(C::BQ_EMPTY));
+            }
+            const int i = x.qb * 32 + (r >> 2);
+            const float2 rec = p.ld[(((long long)x.b * p.Hkv + x.kvh) * p.Tp + x.qb * 32) * 4 + r];
+            const float lse2 = rec.x, Dv = rec.y;
+            for (int j = 0; j < x.n && ok; ++j, ++g) {
+                const int bb = g & 1;
+                ok = warp_wait(bar(C::BS_FULL + bb), (g >> 1) & 1, ab);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t s[32], d[32], pk[16];
+                const uint32_t ts = tmem + lane_base + C::kColBuf + bb * C::kBufStride + 32 * grp;
+                tmem_ld32(ts, s);
+                tmem_ld32(ts + kN, d);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BS_FREE + bb));   // the scores are in registers
+                const int hi = i - j * kN - 32 * grp;                // visible columns e <= hi
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float p0 = ex2(fmaf(__uint_as_float(s[e]), p.sl2, -lse2));
+                    float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), p.sl2, -lse2));
+                    p0 = (e <= hi) ? p0 : 0.f;
+                    p1 = (e + 1 <= hi) ? p1 : 0.f;
+                    pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(d[e]) - Dv), p1 * (__uint_as_float(d[e + 1]) - Dv));
+                }
+                // the previous tile's dQ MMA has read the dS tile
+                ok = warp_wait(bar(C::BDS_FREE), (g & 1) ^ 1u, ab);
+                if (!ok) break;
+                sts_row_chunks(sbase + C::kOffDS, r, 4 * grp, pk);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BDS_READY));
+            }
+            if (!ok || grp != 0) continue;
+            // ---- epilogue of the unit (warps 4-7): dq, dw_q
+            ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
+            if (!ok) break;
+            tc_fence_after();
+            const bool valid = i < p.T;
+            const long long off = valid ? (((long long)x.b * p.T + i) * p.Hq + x.kvh * 4 + (r & 3)) * kD : 0;
+            norm_rope_backward<R>(tmem + lane_base + C::kColDQ, p.scale, p.x + off, valid, w, p.eps, i, p.theta,
+                                  p.dx + off, dwacc);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::BACC_FREE));
+        }
+        if (grp == 0) {
+            float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================ dk/dv kernel
+// Key-stationary (M = 128 keys of one KV head).  Per 64-row query chunk (16
+// tokens x 4 heads): S^T = K~ Q~^T and dP^T = V dA^T into one of two TMEM
+// buffers; eight warps (two per TMEM lane quarter, each taking 32 of the 64
+// columns) load them, release the buffer at once, and write P^T and dS^T as
+// bf16 into shared memory, from where dV += P^T dA and dK~ += dS^T Q~ read
+// them.  So the next chunk's scores are computed while this chunk's
+// probabilities are formed, and every contraction runs at N >= 64 from
+// shared memory.  The same eight warps run the epilogue: dv (warps 4-7),
+// dk through RoPE^T and the RMSNorm backward (warps 8-11).
+struct KvCfg {
+    static constexpr int kM = 64;                    // query rows per chunk (16 tokens x 4 heads)
+    static constexpr int kChTok = 16;
+    static constexpr int kStages = 3;
+    static constexpr uint32_t kKHalf = 128 * kHalfRowBytes;   // 16 KiB
+    static constexpr uint32_t kKTile = 2 * kKHalf;
+    static constexpr uint32_t kCHalf = kM * kHalfRowBytes;    // 8 KiB
+    static constexpr uint32_t kCTile = 2 * kCHalf;
+    static constexpr uint32_t kRecBytes = kM * 8;             // {lse log2 e, D} per row
+    static constexpr uint32_t kStageBytes = 2 * kCTile + 1024;   // Q~ chunk, dA chunk, records
+    static constexpr uint32_t kPTile = 128 * kHalfRowBytes;   // P^T or dS^T: 128 keys x 64 rows bf16
+    static constexpr uint32_t kOffK = 0;
+    static constexpr uint32_t kOffV = kOffK + kKTile;
+    static constexpr uint32_t kOffCh = kOffV + kKTile;
+    static constexpr uint32_t kOffP = kOffCh + kStages * kStageBytes;
+    static constexpr uint32_t kOffDS = kOffP + kPTile;
+    static constexpr uint32_t kOffW = kOffDS + kPTile;
+    static constexpr uint32_t kOffBar = kOffW + 512;
+    static constexpr int kNumBars = 24;
+    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+    // TMEM columns: two {S^T, dP^T} buffers, dV, dK~
+    static constexpr uint32_t kColBuf = 0, kBufStride = 128, kColDV = 256, kColDK = 384;
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
     static constexpr int BKV_FULL = 0, BKV_EMPTY = 1, BCH_FULL = 2, BCH_EMPTY = BCH_FULL + kStages,
-                         BS_FULL = BCH_EMPTY + kStages, BP_READY = BS_FULL + 2, BS_FREE = BP_READY + 2,
-                         BACC_FULL = BS_FREE + 2, BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1;
+                         BS_FULL = BCH_EMPTY + kStages, BS_FREE = BS_FULL + 2, BPS_READY = BS_FREE + 2,
+                         BPS_FREE = BPS_READY + 1, BACC_FULL = BPS_FREE + 1, BACC_FREE = BACC_FULL + 1,
+                         B_DRAIN = BACC_FREE + 1;
     static_assert(B_DRAIN < kNumBars, "barrier count");
 };
 
@@ -755,11 +1059,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(C::BS_FULL + i), 1);
-            mbar_init(bar(C::BP_READY + i), 4);
-            mbar_init(bar(C::BS_FREE + i), 1);
+            mbar_init(bar(C::BS_FREE + i), 8);
         }
+        mbar_init(bar(C::BPS_READY), 8);
+        mbar_init(bar(C::BPS_FREE), 1);
         mbar_init(bar(C::BACC_FULL), 1);
-        mbar_init(bar(C::BACC_FREE), 4);
+        mbar_init(bar(C::BACC_FREE), 8);
         mbar_init(bar(C::B_DRAIN), 1);
         fence_barrier_init();
         tma_prefetch_desc(&tm_k);
@@ -799,7 +1104,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     ok = mbar_wait(bar(C::BCH_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
                     if (!ok) break;
                     const int t0 = 128 * x.kt + C::kChTok * j;
-                    mbar_arrive_expect_tx(bar(C::BCH_FULL + st), 2 * C::kCTile + kM * 8);
+                    mbar_arrive_expect_tx(bar(C::BCH_FULL + st), 2 * C::kCTile + C::kRecBytes);
                     for (int h = 0; h < 2; ++h) {
                         tma_load_4d(stage(st) + h * C::kCHalf, &tm_q, bar(C::BCH_FULL + st), h * 64, x.kvh * 4, t0,
                                     x.b);
@@ -807,7 +1112,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                     x.kvh * 4, t0, x.b);
                     }
                     bulk_load(stage(st) + 2 * C::kCTile, p.ld + (((long long)x.b * p.Hkv + x.kvh) * p.Tp + t0) * 4,
-                              kM * 8, bar(C::BCH_FULL + st));
+                              C::kRecBytes, bar(C::BCH_FULL + st));
                 }
             }
             for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
@@ -823,14 +1128,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ws.init(p);
             wd.init(p);
             int ns = 0, nd = 0;
-            uint64_t t_last = globaltimer();
+            PollWatch watch;
             while (wd.valid) {
                 bool progressed = false;
                 if (ws.valid && ns < nd + 2 && mbar_test(bar(C::BKV_FULL), ws.k & 1) &&
                     mbar_test(bar(C::BCH_FULL + ns % kStages), (ns / kStages) & 1) &&
                     mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
                     tc_fence_after();
-                    const uint32_t dS = tmem + (ns & 1) * 128;
+                    const uint32_t dS = tmem + C::kColBuf + (ns & 1) * C::kBufStride;
                     const uint32_t qs = stage(ns % kStages), as = qs + C::kCTile;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -852,45 +1157,39 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     ++ns;
                     progressed = true;
                 }
-                if (nd < ns && mbar_test(bar(C::BP_READY + (nd & 1)), (nd >> 1) & 1) &&
+                if (nd < ns && mbar_test(bar(C::BPS_READY), nd & 1) &&
                     (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
                     tc_fence_after();
-                    const uint32_t pt = tmem + (nd & 1) * 128;
                     const uint32_t qs = stage(nd % kStages), as = qs + C::kCTile;
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
-                        mma_ts(tmem + C::kColDV, pt + kk * 8, smem_desc_sw128(as + kk * 16 * 128, C::kCHalf, 1024),
-                               idesc_acc, (wd.j > 0 || kk > 0));
+                        mma_ss(tmem + C::kColDV, smem_desc_sw128(sbase + C::kOffP + kk * 32, 16, 1024),
+                               smem_desc_sw128(as + kk * 16 * 128, C::kCHalf, 1024), idesc_acc, (wd.j > 0 || kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
-                        mma_ts(tmem + C::kColDK, pt + kM + kk * 8,
+                        mma_ss(tmem + C::kColDK, smem_desc_sw128(sbase + C::kOffDS + kk * 32, 16, 1024),
                                smem_desc_sw128(qs + kk * 16 * 128, C::kCHalf, 1024), idesc_acc, (wd.j > 0 || kk > 0));
                     mma_commit(bar(C::BCH_EMPTY + nd % kStages));
-                    mma_commit(bar(C::BS_FREE + (nd & 1)));
+                    mma_commit(bar(C::BPS_FREE));
                     if (wd.last()) mma_commit(bar(C::BACC_FULL));
                     wd.next(p);
                     ++nd;
                     progressed = true;
                 }
-                if (progressed) {
-                    t_last = globaltimer();
-                } else {
-                    if (ab.raised()) break;
-                    if (globaltimer() - t_last > kWaitLimitNs) {
-                        ab.raise(kStatusTimeout);
-                        break;
-                    }
-                }
+                if (!watch.tick(progressed, ab)) break;
             }
             mma_commit(bar(C::B_DRAIN));
             drain_wait(bar(C::B_DRAIN), 0);
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
-        // ================================================= P^T, dS^T
-        const int r = tid - 128;   // key of the tile
+    } else if (warp >= 4) {
+        // ================================================= P^T, dS^T (8 warps) and the epilogue
+        const int grp = (warp - 4) >> 2;           // column half of each chunk: rows 32 grp .. 32 grp + 31
+        const int r = 32 * (warp & 3) + lane;      // key of the tile (TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
         const int W = kSwa ? p.window : (1 << 30);
+        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
         bool ok = true;
         int g = 0;
         KUnit x;
@@ -904,88 +1203,85 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (ok) ok = warp_wait(bar(C::BCH_FULL + st), (g / kStages) & 1, ab);
                 if (!ok) break;
                 tc_fence_after();
-                const int t0 = 128 * x.kt + C::kChTok * j;
-                const int lo = jkey - t0, hi = jkey - t0 + W - 1;   // visible chunk tokens
-                const uint32_t ts = tmem + lane_base + bb * 128;
-                const uint32_t rec = stage(st) + 2 * C::kCTile;
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t s[32], d[32], pk[16], dk[16];
-                    tmem_ld32(ts + 32 * hf, s);
-                    tmem_ld32(ts + kM + 32 * hf, d);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        // records of rows 32 hf + e .. + 3 (one token, four heads)
-                        const uint4 ra = lds128(rec + (32 * hf + e) * 8);
-                        const uint4 rb = lds128(rec + (32 * hf + e + 2) * 8);
-                        const float l2[4] = {__uint_as_float(ra.x), __uint_as_float(ra.z), __uint_as_float(rb.x),
-                                             __uint_as_float(rb.z)};
-                        const float dv[4] = {__uint_as_float(ra.y), __uint_as_float(ra.w), __uint_as_float(rb.y),
-                                             __uint_as_float(rb.w)};
-                        const int tok = (32 * hf + e) >> 2;
-                        const bool vis = tok >= lo && tok <= hi;
-                        float pp[4], ds[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            pp[q] = vis ? ex2(fmaf(__uint_as_float(s[e + q]), p.sl2, -l2[q])) : 0.f;
-                            ds[q] = pp[q] * (__uint_as_float(d[e + q]) - dv[q]);
-                        }
-                        pk[e >> 1] = pack_bf16(pp[0], pp[1]);
-                        pk[(e >> 1) + 1] = pack_bf16(pp[2], pp[3]);
-                        dk[e >> 1] = pack_bf16(ds[0], ds[1]);
-                        dk[(e >> 1) + 1] = pack_bf16(ds[2], ds[3]);
-                    }
-                    tmem_st16(ts + 16 * hf, pk);
-                    tmem_st16(ts + kM + 16 * hf, dk);
-                }
-                tmem_wait_st();
+                uint32_t s[32], d[32];
+                const uint32_t ts = tmem + lane_base + C::kColBuf + bb * C::kBufStride + 32 * grp;
+                tmem_ld32(ts, s);
+                tmem_ld32(ts + kM, d);
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::BP_READY + bb));
+                if (lane == 0) mbar_arrive(bar(C::BS_FREE + bb));   // the scores are in registers
+                const int t0 = 128 * x.kt + C::kChTok * j;
+                const int lo = jkey - t0, hi = jkey - t0 + W - 1;   // visible chunk tokens
+                const uint32_t rec = stage(st) + 2 * C::kCTile + 32 * grp * 8;
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    // records of rows 32 grp + e .. + 3 (one token, four heads)
+                    const uint4 ra = lds128(rec + e * 8);
+                    const uint4 rb = lds128(rec + (e + 2) * 8);
+                    const float l2[4] = {__uint_as_float(ra.x), __uint_as_float(ra.z), __uint_as_float(rb.x),
+                                         __uint_as_float(rb.z)};
+                    const float dv[4] = {__uint_as_float(ra.y), __uint_as_float(ra.w), __uint_as_float(rb.y),
+                                         __uint_as_float(rb.w)};
+                    const int tok = (32 * grp + e) >> 2;
+                    const bool vis = tok >= lo && tok <= hi;
+                    float pp[4], ds[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        pp[q] = vis ? ex2(fmaf(__uint_as_float(s[e + q]), p.sl2, -l2[q])) : 0.f;
+                        ds[q] = pp[q] * (__uint_as_float(d[e + q]) - dv[q]);
+                    }
+                    pk[e >> 1] = pack_bf16(pp[0], pp[1]);
+                    pk[(e >> 1) + 1] = pack_bf16(pp[2], pp[3]);
+                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                    dk[(e >> 1) + 1] = pack_bf16(ds[2], ds[3]);
+                }
+                // the previous chunk's dV/dK have read the P^T / dS^T tiles
+                ok = warp_wait(bar(C::BPS_FREE), (g & 1) ^ 1u, ab);
+                if (!ok) break;
+                sts_row_chunks(sbase + C::kOffP, r, 4 * grp, pk);
+                sts_row_chunks(sbase + C::kOffDS, r, 4 * grp, dk);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BPS_READY));
             }
-        }
-    } else if (warp >= 8) {
-        // ================================================= epilogue: dv, dk, dw_k
-        const int r = tid - 256;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
-        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
-        bool ok = true;
-        KUnit x;
-        for (int k = 0; k < nunits && ok; ++k) {
-            kv_unit_at<kSwa>(p, k, x);
+            if (!ok) break;
+            // ---- epilogue of the unit: dv (warps 4-7), dk and dw_k (warps 8-11)
             ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
             if (!ok) break;
             tc_fence_after();
-            const int jkey = 128 * x.kt + r;
             const bool valid = jkey < p.T;
             const long long off = valid ? (((long long)x.b * p.T + jkey) * p.Hkv + x.kvh) * kD : 0;
-            // dv = sum_i P_ij dA_i
+            if (grp == 0) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + C::kColDV + 32 * c, v);
-                tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + C::kColDV + 32 * c, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 o = make_uint4(
-                        pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1])),
-                        pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                        pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                        pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-                    if (valid) reinterpret_cast<uint4 *>(p.dv + off)[4 * c + q] = o;
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 o = make_uint4(
+                            pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1])),
+                            pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                            pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                            pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+                        if (valid) reinterpret_cast<uint4 *>(p.dv + off)[4 * c + q] = o;
+                    }
                 }
+            } else {
+                norm_rope_backward<R>(tmem + lane_base + C::kColDK, p.scale, p.x + off, valid, w, p.eps, jkey,
+                                      p.theta, p.dx + off, dwacc);
             }
-            norm_rope_backward<R>(tmem + lane_base + C::kColDK, p.scale, p.x + off, valid, w, p.eps, jkey,
-                                  p.theta, p.dx + off, dwacc);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::BACC_FREE));
         }
-        float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
+        if (grp == 1) {
+            float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
+            for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
+        }
     }
 
     tc_fence_before();

@@ -227,7 +227,7 @@ full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int kq = 0, ns = 0, npv = 0;
             Unit xq;
             bool q_more = unit_at(p, 0, xq);
-            uint64_t t_last = globaltimer();
+            PollWatch watch;
             while (wp.valid) {
                 bool progressed = false;
                 if (q_more && mbar_test(bar(BQ_EMPTY + (kq & 1)), ((kq >> 1) & 1) ^ 1u)) {
@@ -274,15 +274,7 @@ full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++npv;
                     progressed = true;
                 }
-                if (progressed) {
-                    t_last = globaltimer();
-                } else {
-                    if (ab.raised()) break;
-                    if (globaltimer() - t_last > kWaitLimitNs) {
-                        ab.raise(kStatusTimeout);
-                        break;
-                    }
-                }
+                if (!watch.tick(progressed, ab)) break;
             }
             mma_commit(bar(B_DRAIN));
             drain_wait(bar(B_DRAIN), 0);

@@ -50,7 +50,7 @@ bool set_bwd_smem()
 {
     using namespace gswa::bwd;
     return set_smem(bwd_dq_kernel<R, true>, DqCfg<true>::kSmemBytes) ||
-           set_smem(bwd_dq_kernel<R, false>, DqCfg<false>::kSmemBytes) ||
+           set_smem(bwd_dq_full_kernel<R>, DqFullCfg::kSmemBytes) ||
            set_smem(bwd_dkdv_kernel<R, true>, KvCfg::kSmemBytes) ||
            set_smem(bwd_dkdv_kernel<R, false>, KvCfg::kSmemBytes);
 }
@@ -265,7 +265,10 @@ void launch_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::
                      unsigned gk, cudaStream_t st)
 {
     using namespace gswa::bwd;
-    bwd_dq_kernel<R, kSwa><<<gq, kThreads, DqCfg<kSwa>::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
+    if constexpr (kSwa)
+        bwd_dq_kernel<R, true><<<gq, kThreads, DqCfg<true>::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
+    else
+        bwd_dq_full_kernel<R><<<gq, kThreads, DqFullCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
     bwd_dkdv_kernel<R, kSwa><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
 }
 

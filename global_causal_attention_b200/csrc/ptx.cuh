@@ -127,6 +127,35 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
     }
 }
 
+// Stall watchdog of a polling loop (a thread that tests several barriers in
+// turn): call tick(progressed) once per pass.  The wall clock is a slow read,
+// so it is consulted only every 512 idle passes.  Returns false (with the
+// CTA's abort flag raised) once the loop has made no progress for
+// kWaitLimitNs, or when another role raised the flag.
+struct PollWatch {
+    uint32_t idle = 0;
+    uint64_t t0 = 0;
+    __device__ __forceinline__ bool tick(bool progressed, const Abort &ab)
+    {
+        if (progressed) {
+            idle = 0;
+            return true;
+        }
+        if ((++idle & 511u) != 0) return true;
+        if (ab.raised()) return false;
+        const uint64_t now = globaltimer();
+        if (idle == 512u) {
+            t0 = now;
+            return true;
+        }
+        if (now - t0 > kWaitLimitNs) {
+            ab.raise(kStatusTimeout);
+            return false;
+        }
+        return true;
+    }
+};
+
 // Warp-uniform wait: every lane waits (and so acquires) itself, then the warp
 // agrees, so a wait that gave up in one lane stops the whole warp.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Abort &ab)

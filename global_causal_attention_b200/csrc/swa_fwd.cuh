@@ -476,7 +476,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             wp.init(p, u0);
             wq.init(p, u0);
             int ns = 0, npv = 0, nq = 0;
-            uint64_t t_last = globaltimer();
+            PollWatch watch;
             while (npv < n) {
                 bool progressed = false;
                 // Q tile of unit nq into slot nq & 1 once S(nq - 2) has consumed it
@@ -546,15 +546,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         progressed = true;
                     }
                 }
-                if (progressed) {
-                    t_last = globaltimer();
-                } else {
-                    if (ab.raised()) break;
-                    if (globaltimer() - t_last > kWaitLimitNs) {
-                        ab.raise(kStatusTimeout);
-                        break;
-                    }
-                }
+                if (!watch.tick(progressed, ab)) break;
             }
             // all MMAs issued by this thread complete before TMEM is freed, and
             // every Q load it issued has landed before shared memory is released
