@@ -80,10 +80,7 @@ int device_setup(int *num_sms)
                    set_smem(gswa::swa::swa_fwd_kernel<42>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::swa::swa_fwd_kernel<64>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes) ||
-                   set_smem(gswa::full::full_fwd_kernel<0>, gswa::full::kSmemBytes) ||
-                   set_smem(gswa::full::full_fwd_kernel<42>, gswa::full::kSmemBytes) ||
-                   set_smem(gswa::full::full_fwd_kernel<64>, gswa::full::kSmemBytes) ||
-                   set_smem(gswa::full::full_fwd_kernel<128>, gswa::full::kSmemBytes) ||
+                   set_smem(gswa::full::full_fwd_kernel, gswa::full::kSmemBytes) ||
                    set_bwd_smem<0>() || set_bwd_smem<42>() || set_bwd_smem<64>() || set_bwd_smem<128>()) {
             d.status = GSWA_ERR_LAUNCH;
         }
@@ -164,10 +161,16 @@ void fill_dec(gswa::dec::Params &p, const gswa_shape_t *s)
     fill_theta(p.theta, s->rope_dims, s->rope_base);
 }
 
-// Prepared-key workspace of the full causal forward: k~ [B, T, Hkv, D] bf16.
-size_t full_fwd_ws(const gswa_shape_t *s)
+// Workspace of the full causal forward: prepared keys k~ [B, T, Hkv, D] then
+// prepared queries q~ [B, T, Hq, D], bf16.
+size_t full_fwd_ws_keys(const gswa_shape_t *s)
 {
     return align256((size_t)s->B * s->T * s->Hkv * s->D * 2);
+}
+
+size_t full_fwd_ws(const gswa_shape_t *s)
+{
+    return full_fwd_ws_keys(s) + align256((size_t)s->B * s->T * s->Hq * s->D * 2);
 }
 
 // RMSNorm + partial RoPE of x [B, T, H, 128] into out, positions pos0 + t.
@@ -487,14 +490,16 @@ int full_attn_fwd(const gswa_shape_t *s, const void *q, const void *k, const voi
     if (rc != GSWA_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // prepared keys once, into the workspace
-    rc = launch_qk_prep(s, s->Hkv, k, w_k, workspace, 0, st, num_sms);
+    // prepared keys and queries once, into the workspace
+    void *kt = workspace;
+    void *qt = static_cast<char *>(workspace) + full_fwd_ws_keys(s);
+    rc = launch_qk_prep(s, s->Hkv, k, w_k, kt, 0, st, num_sms);
+    if (rc == GSWA_OK) rc = launch_qk_prep(s, s->Hq, q, w_q, qt, 0, st, num_sms);
     if (rc != GSWA_OK) return rc;
 
-    CUtensorMap tq, tk, tv, ty;
-    if (encode_bthd(&tq, q, s->B, s->T, s->Hq, s->D, 4, 32) ||
-        encode_bthd(&ty, y, s->B, s->T, s->Hq, s->D, 4, 32) ||
-        encode_bthd(&tk, workspace, s->B, s->T, s->Hkv, s->D, 1, 128) ||
+    CUtensorMap tq, tk, tv;
+    if (encode_bthd(&tq, qt, s->B, s->T, s->Hq, s->D, 4, 32) ||
+        encode_bthd(&tk, kt, s->B, s->T, s->Hkv, s->D, 1, 128) ||
         encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, 128))
         return GSWA_ERR_INVALID_ARG;
 
@@ -507,21 +512,14 @@ int full_attn_fwd(const gswa_shape_t *s, const void *q, const void *k, const voi
     p.nq = (s->T + gswa::full::kTok - 1) / gswa::full::kTok;
     p.nkt = (s->T + gswa::full::kKeys - 1) / gswa::full::kKeys;
     p.units = (long long)s->B * s->Hkv * p.nq;
-    p.eps = s->eps;
     p.sl2 = s->scale * 1.4426950408889634f;
     p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.y = static_cast<__nv_bfloat16 *>(y);
     p.lse = lse;
-    fill_theta(p.theta, s->rope_dims, s->rope_base);
 
     const long long grid = p.units < num_sms ? p.units : num_sms;
-    const dim3 gr((unsigned)grid), bl(gswa::full::kThreads);
-    const uint32_t sm = gswa::full::kSmemBytes;
-    switch (s->rope_dims) {
-    case 0: gswa::full::full_fwd_kernel<0><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
-    case 42: gswa::full::full_fwd_kernel<42><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
-    case 64: gswa::full::full_fwd_kernel<64><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
-    default: gswa::full::full_fwd_kernel<128><<<gr, bl, sm, st>>>(tq, tk, tv, ty, p); break;
-    }
+    gswa::full::full_fwd_kernel<<<(unsigned)grid, gswa::full::kThreads, gswa::full::kSmemBytes, st>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 

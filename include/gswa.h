@@ -95,7 +95,8 @@ int gswa_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void
  * layers attend over the whole context and drop the gate).  Same layouts
  * as gswa_fwd without g; shape->window is ignored.  Needs a workspace of
  * gswa_workspace_bytes(GSWA_OP_FULL_FWD) bytes (device, 16-byte aligned):
- * it receives the prepared keys.
+ * it receives the prepared keys and queries (each key tile is reused by
+ * every later query block, so it is normed and rotated once).
  */
 int full_attn_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                   const void *w_q, const void *w_k, void *y, float *lse, void *workspace,

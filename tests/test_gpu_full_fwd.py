@@ -44,14 +44,40 @@ def test_full_fwd_matches_oracle(name):
     assert_fwd_close(lse, lo, "lse")
 
 
-@pytest.mark.parametrize("R", [0, 42])
-def test_full_fwd_running_max_rescale(R):
+def spiky_weights():
+    """Norm weights of 1 except one dimension of 4 in each: the score bound
+    D max|w_q| max|w_k| scale log2 e (about 270) is past the range where the kernel
+    uses it as a fixed softmax reference, so the running-max path runs, while the
+    scores themselves stay close to those of unit weights."""
+    wq, wk = torch.ones(128), torch.ones(128)
+    wq[5] = 4.0
+    wk[77] = 4.0
+    return wq.to(torch.bfloat16), wk.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("name", ["tiny_512", "ragged_200_gqa2", "T1024_many_tiles", "T33"])
+def test_full_fwd_running_max_path(name):
+    s, seed, _ = CASES[name]
+    x = attention_inputs(s, seed)
+    x["wq"], x["wk"] = spiky_weights()
+    y, lse = run_gpu(s, x)
+    yo, lo = oracle.attn_fwd(x["q"], x["k"], x["v"], None, x["wq"], x["wk"], window=0, gated=False,
+                             **oracle.shape_kwargs(s))
+    assert_fwd_close(y, yo, "y")
+    assert_fwd_close(lse, lo, "lse")
+
+
+@pytest.mark.parametrize("R,spiky", [(0, False), (42, False), (42, True)])
+def test_full_fwd_running_max_rescale(R, spiky):
     """Every query equals a vector u; keys before position 128 equal -u and later
     keys +u.  For rows past 128 the second key tile's scores exceed the first
-    tile's max by ~15 (natural units), far past the 2^8 threshold, so the O
-    accumulator is rescaled in TMEM."""
+    tile's max by ~15 (natural units), far past the 2^8 threshold: with spiky
+    norm weights (running-max path) the O accumulator is rescaled in TMEM; with
+    unit weights the fixed reference covers the whole range."""
     s = Shape(B=1, T=700, Hq=4, Hkv=1, rope_dims=R)
     x = attention_inputs(s, 14)
+    if spiky:
+        x["wq"], x["wk"] = spiky_weights()
     u = randn_bf16((128,), 15)
     x["q"] = u.expand(s.B, s.T, s.Hq, 128).contiguous()
     k = u.expand(s.B, s.T, s.Hkv, 128).contiguous().clone()
