@@ -10,10 +10,13 @@
 //   full_decode: linear cache [B, Hkv, Tmax, D], split over the cache length:
 //     a prologue prepares q~ (f32, into the workspace) and appends k~, v; a
 //     chunk kernel computes, per 4096-key chunk, the partial (max, sum, O) of
-//     the 4 query heads (lanes = keys for q.k with q~ broadcast from shared
-//     memory, lanes = dims for P V with 8-byte coalesced value loads); a
-//     combine kernel merges the chunks by their log-sum-exp weights.
+//     the 4 query heads from K/V rows streamed by TMA through a shared-memory
+//     ring (lanes = keys for q.k with q~ broadcast from shared memory, lanes =
+//     dims for P V); a combine kernel merges the chunks by their log-sum-exp
+//     weights.
 #pragma once
+
+#include <cuda.h>
 
 #include "ptx.cuh"
 #include "swa_fwd.cuh"
@@ -226,9 +229,29 @@ __device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t x, float s)
 
 // Chunk c of (b, kvh): partial softmax state of the 4 heads over keys
 // [c * kChunk, (c + 1) * kChunk) intersected with [0, pos].
-__global__ void __launch_bounds__(kChunkWarps * 32)
-full_decode_chunk_kernel(const __grid_constant__ Params p)
+//
+// The chunk's K and V rows stream through a ring of kDecStages shared-memory
+// stages of kStageKeys keys, loaded by TMA (128-byte swizzle, so a lane per
+// key reads its row without bank conflicts) by a producer warp; compute warp
+// w takes stages w, w + kChunkWarps, ... and keeps its own running (max, sum,
+// O) per head, merged at the end.  The loads of many stages are in flight at
+// once, which is what keeps HBM busy.
+constexpr int kStageKeys = 32;
+constexpr int kDecStages = 12;
+constexpr uint32_t kDecHalf = kStageKeys * 128;          // 32 keys x 64 dims bf16: 4 KiB
+constexpr uint32_t kDecTile = 2 * kDecHalf;               // one operand of a stage: 8 KiB
+constexpr uint32_t kDecStageBytes = 2 * kDecTile;          // K and V
+constexpr uint32_t kDecOffBar = kDecStages * kDecStageBytes;
+constexpr uint32_t kDecSmemBytes = kDecOffBar + 2 * kDecStages * 8 + 4 + 1024;
+constexpr int kChunkThreads = (kChunkWarps + 1) * 32;     // compute warps + the producer warp
+
+__global__ void __launch_bounds__(kChunkThreads, 1)
+full_decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ Params p)
 {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
     __shared__ __align__(16) float qt[4][kD];
     __shared__ float wm[kChunkWarps][4], wl[kChunkWarps][4];
     __shared__ __align__(16) float wo[kChunkWarps][4][kD];
@@ -237,84 +260,128 @@ full_decode_chunk_kernel(const __grid_constant__ Params p)
     const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
     const long long pos = p.pos[b];
     if (pos < 0 || pos >= p.Tmax || (long long)c * kChunk > pos) return;   // nothing to attend here
+    auto full = [&](int st) -> uint32_t { return sbase + kDecOffBar + 8u * st; };
+    auto empty = [&](int st) -> uint32_t { return sbase + kDecOffBar + 8u * (kDecStages + st); };
+    Abort ab{reinterpret_cast<volatile int *>(smem + kDecOffBar + 16 * kDecStages)};
+    if (threadIdx.x == 0) {
+        *ab.flag = 0;
+        for (int i = 0; i < kDecStages; ++i) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), 1);
+        }
+        fence_barrier_init();
+    }
     for (int i = threadIdx.x; i < 4 * kD; i += blockDim.x)
         qt[i / kD][i % kD] = p.qt[((long long)b * p.Hq + kvh * 4) * kD + i];
     __syncthreads();
-    const long long rowbase = ((long long)b * p.Hkv + kvh) * p.Tmax;
     const long long k0 = (long long)c * kChunk;
     const long long k1 = min(k0 + kChunk, pos + 1);   // exclusive end
-    const int per_warp = kChunk / kChunkWarps;
-    const long long w0 = k0 + (long long)warp * per_warp;
-    const long long w1 = min(w0 + per_warp, k1);
+    const int nst = (int)((k1 - k0 + kStageKeys - 1) / kStageKeys);
+    const int row0 = (int)(((long long)b * p.Hkv + kvh) * p.Tmax + k0);   // first cache row of the chunk
 
-    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running max (log2 units)
-    float l[4] = {0.f, 0.f, 0.f, 0.f};                          // this lane's keys' sums
-    uint64_t o[4][2];                                           // dims 4 lane..+3, as 2 pairs
-#pragma unroll
-    for (int h = 0; h < 4; ++h) o[h][0] = o[h][1] = 0;
-    for (long long t0 = w0; t0 < w1; t0 += 32) {
-        const long long key = t0 + lane;
-        float s[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (key < w1) {
-            const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + (rowbase + key) * kD);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int ch = 0; ch < 16; ++ch) {
-                const uint4 kv = kr[ch];
-                const float2 ka = unpack_bf16(kv.x), kb = unpack_bf16(kv.y), kc2 = unpack_bf16(kv.z),
-                             kd = unpack_bf16(kv.w);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float4 qa = *reinterpret_cast<const float4 *>(&qt[h][8 * ch]);
-                    const float4 qb = *reinterpret_cast<const float4 *>(&qt[h][8 * ch + 4]);
-                    float a = acc[h];
-                    a = fmaf(qa.x, ka.x, fmaf(qa.y, ka.y, fmaf(qa.z, kb.x, fmaf(qa.w, kb.y, a))));
-                    a = fmaf(qb.x, kc2.x, fmaf(qb.y, kc2.y, fmaf(qb.z, kd.x, fmaf(qb.w, kd.y, a))));
-                    acc[h] = a;
+    if (warp == kChunkWarps) {
+        // ================================================= producer
+        if (lane == 0) {
+            bool ok = true;
+            int s = 0;
+            for (; s < nst && ok; ++s) {
+                const int st = s % kDecStages;
+                ok = mbar_wait(empty(st), ((s / kDecStages) & 1) ^ 1u, ab);
+                if (!ok) break;
+                mbar_arrive_expect_tx(full(st), kDecStageBytes);
+                const uint32_t dst = sbase + st * kDecStageBytes;
+                const int row = row0 + s * kStageKeys;
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_2d(dst + h * kDecHalf, &tm_k, full(st), h * 64, row);
+                    tma_load_2d(dst + kDecTile + h * kDecHalf, &tm_v, full(st), h * 64, row);
                 }
             }
-#pragma unroll
-            for (int h = 0; h < 4; ++h) s[h] = acc[h] * p.sl2;
+            // no copy may still be landing when the CTA exits
+            const uint64_t t0 = globaltimer();
+            for (int i = (s > kDecStages ? s - kDecStages : 0); i < s; ++i)
+                while (!mbar_try_wait(full(i % kDecStages), (i / kDecStages) & 1))
+                    if (globaltimer() - t0 > 200000000ull) break;
         }
-        float pr[4], alpha[4];
+    } else {
+        // ================================================= compute warps
+        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running max (log2 units)
+        float l[4] = {0.f, 0.f, 0.f, 0.f};                          // this lane's keys' sums
+        uint64_t o[4][2];                                           // dims 4 lane..+3, as 2 pairs
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const float tm = warp_max(s[h]);
-            const float mn = fmaxf(m[h], tm);
-            alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
-            m[h] = mn;
-            pr[h] = (s[h] == -INFINITY) ? 0.f : ex2(s[h] - mn);
-            l[h] = l[h] * alpha[h] + pr[h];
-            const uint64_t a2 = f2_bits(alpha[h], alpha[h]);
-            asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][0]) : "l"(a2));
-            asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][1]) : "l"(a2));
-        }
-        const int nk = (int)min((long long)32, w1 - t0);
-        for (int j = 0; j < nk; ++j) {
-            const uint2 vv = *reinterpret_cast<const uint2 *>(p.vc + (rowbase + t0 + j) * kD + 4 * lane);
-            const float2 va = unpack_bf16(vv.x), vb = unpack_bf16(vv.y);
-            const uint64_t v01 = f2_bits(va.x, va.y), v23 = f2_bits(vb.x, vb.y);
+        for (int h = 0; h < 4; ++h) o[h][0] = o[h][1] = 0;
+        // V row j, dims 4 lane .. 4 lane + 3: half lane / 16, 16-byte chunk (lane % 16) / 2, 8-byte word lane % 2
+        const uint32_t v_half = (uint32_t)(lane >> 4) * kDecHalf, v_chunk = (uint32_t)((lane & 15) >> 1),
+                       v_word = (uint32_t)(lane & 1) * 8;
+        for (int s = warp; s < nst; s += kChunkWarps) {
+            const int st = s % kDecStages;
+            if (!warp_wait(full(st), (s / kDecStages) & 1, ab)) break;
+            const uint32_t ks = sbase + st * kDecStageBytes, vs = ks + kDecTile;
+            const long long t0 = k0 + (long long)s * kStageKeys;
+            const int nk = (int)min((long long)kStageKeys, k1 - t0);
+            float sc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (lane < nk) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int ch = 0; ch < 16; ++ch) {
+                    const uint4 kv = lds128(ks + swa::chunk_off(lane, ch, kDecHalf));
+                    const float2 ka = unpack_bf16(kv.x), kb = unpack_bf16(kv.y), kc2 = unpack_bf16(kv.z),
+                                 kd = unpack_bf16(kv.w);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float4 qa = *reinterpret_cast<const float4 *>(&qt[h][8 * ch]);
+                        const float4 qb = *reinterpret_cast<const float4 *>(&qt[h][8 * ch + 4]);
+                        float a = acc[h];
+                        a = fmaf(qa.x, ka.x, fmaf(qa.y, ka.y, fmaf(qa.z, kb.x, fmaf(qa.w, kb.y, a))));
+                        a = fmaf(qb.x, kc2.x, fmaf(qb.y, kc2.y, fmaf(qb.z, kd.x, fmaf(qb.w, kd.y, a))));
+                        acc[h] = a;
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < 4; ++h) sc[h] = acc[h] * p.sl2;
+            }
+            float pr[4], alpha[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                const float ps = __shfl_sync(0xffffffffu, pr[h], j);
-                ffma2(o[h][0], v01, ps);
-                ffma2(o[h][1], v23, ps);
+                const float tm = warp_max(sc[h]);
+                const float mn = fmaxf(m[h], tm);
+                alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+                m[h] = mn;
+                pr[h] = (sc[h] == -INFINITY) ? 0.f : ex2(sc[h] - mn);
+                l[h] = l[h] * alpha[h] + pr[h];
+                const uint64_t a2 = f2_bits(alpha[h], alpha[h]);
+                asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][0]) : "l"(a2));
+                asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(o[h][1]) : "l"(a2));
             }
-        }
-    }
-    // combine the warps of this chunk
+            for (int j = 0; j < nk; ++j) {
+                const uint32_t va = vs + v_half + (uint32_t)j * 128 + ((v_chunk ^ (uint32_t)(j & 7)) << 4) + v_word;
+                uint32_t v0, v1;
+                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(va));
+                const float2 fa = unpack_bf16(v0), fb = unpack_bf16(v1);
+                const uint64_t v01 = f2_bits(fa.x, fa.y), v23 = f2_bits(fb.x, fb.y);
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const float lsum = warp_sum(l[h]);
-        if (lane == 0) {
-            wm[warp][h] = m[h];
-            wl[warp][h] = lsum;
+                for (int h = 0; h < 4; ++h) {
+                    const float ps = __shfl_sync(0xffffffffu, pr[h], j);
+                    ffma2(o[h][0], v01, ps);
+                    ffma2(o[h][1], v23, ps);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(st));
         }
-        float2 a = *reinterpret_cast<float2 *>(&o[h][0]), bq = *reinterpret_cast<float2 *>(&o[h][1]);
-        *reinterpret_cast<float4 *>(&wo[warp][h][4 * lane]) = make_float4(a.x, a.y, bq.x, bq.y);
+        // this warp's state, for the merge
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float lsum = warp_sum(l[h]);
+            if (lane == 0) {
+                wm[warp][h] = m[h];
+                wl[warp][h] = lsum;
+            }
+            float2 a = *reinterpret_cast<float2 *>(&o[h][0]), bq = *reinterpret_cast<float2 *>(&o[h][1]);
+            *reinterpret_cast<float4 *>(&wo[warp][h][4 * lane]) = make_float4(a.x, a.y, bq.x, bq.y);
+        }
     }
     __syncthreads();
-    // thread t: head t / 32... one warp per head: lanes cover dims 4 lane .. +3
+    // one warp per head merges the warps: lanes cover dims 4 lane .. + 3
     if (warp < 4) {
         const int h = warp;
         float M = -INFINITY;

@@ -81,6 +81,7 @@ int device_setup(int *num_sms)
                    set_smem(gswa::swa::swa_fwd_kernel<64>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::full::full_fwd_kernel, gswa::full::kSmemBytes) ||
+                   set_smem(gswa::dec::full_decode_chunk_kernel, gswa::dec::kDecSmemBytes) ||
                    set_bwd_smem<0>() || set_bwd_smem<42>() || set_bwd_smem<64>() || set_bwd_smem<128>()) {
             d.status = GSWA_ERR_LAUNCH;
         }
@@ -113,6 +114,20 @@ int encode_bthd(CUtensorMap *m, const void *base, int B, int T, int H, int D, in
                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
+}
+
+// 2-D bf16 tensor map over `rows` rows of 128 elements (a cache viewed as
+// [B * Hkv * Tmax, 128]) with a {64, box_rows} box and the 128-byte swizzle.
+int encode_rows(CUtensorMap *m, const void *base, long long rows, int box_rows)
+{
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
 }
 
@@ -626,8 +641,16 @@ int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
     p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                        align256((size_t)s->B * s->Hq * s->D * 4));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // cache rows as TMA coordinates (32-bit)
+    CUtensorMap tkc, tvc;
+    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
+    if (cache_rows + gswa::dec::kStageKeys > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (encode_rows(&tkc, k_cache, cache_rows, gswa::dec::kStageKeys) ||
+        encode_rows(&tvc, v_cache, cache_rows, gswa::dec::kStageKeys))
+        return GSWA_ERR_INVALID_ARG;
     gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
-    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkWarps * 32, 0, st>>>(p);
+    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkThreads,
+                                          gswa::dec::kDecSmemBytes, st>>>(tkc, tvc, p);
     gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
@@ -668,8 +691,16 @@ int full_decode_noalloc(const gswa_shape_t *s, const void *q, const void *k, con
     p.qt = static_cast<float *>(scratch);
     p.part = reinterpret_cast<float *>(static_cast<char *>(scratch) + q_bytes);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // cache rows as TMA coordinates (32-bit)
+    CUtensorMap tkc, tvc;
+    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
+    if (cache_rows + gswa::dec::kStageKeys > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (encode_rows(&tkc, k_cache, cache_rows, gswa::dec::kStageKeys) ||
+        encode_rows(&tvc, v_cache, cache_rows, gswa::dec::kStageKeys))
+        return GSWA_ERR_INVALID_ARG;
     gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
-    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkWarps * 32, 0, st>>>(p);
+    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkThreads,
+                                          gswa::dec::kDecSmemBytes, st>>>(tkc, tvc, p);
     gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
