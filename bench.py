@@ -55,8 +55,12 @@ LAUNCHES = {"gswa_fwd": 1, "gswa_bwd": 7, "full_attn_fwd": 2, "full_attn_bwd": 7
 
 # DRAM bytes (read + write) of one call, from an ncu capture of the same
 # launches (dram__bytes_read.sum + dram__bytes_write.sum summed over the
-# call's kernels); None until captured for the current kernels.
-TRAFFIC = {}
+# call's kernels).  Absent entries are reported as null: not captured for the
+# current kernels.
+TRAFFIC = {
+    ("train_4k", "full_attn_bwd"): 9_568_000_000,    # 8.96 GB read + 0.61 GB written, 7 launches
+    ("decode_256k", "full_decode"): 34_430_000_000,  # 34.40 GB read + 0.03 GB written, 3 launches
+}
 
 
 def peaks():
