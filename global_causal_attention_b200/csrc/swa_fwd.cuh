@@ -606,6 +606,24 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int t = r >> 2;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const float ln2 = 0.6931471805599453f;
+        // Softmax reference: the QK norm bounds every raw score by
+        // D max|w_q| max|w_k|, and softmax is shift-invariant, so while that
+        // bound (times scale log2 e, 2 % headroom) is at most 60 it serves as
+        // the reference and the max pass is skipped (no P of a visible key
+        // falls below 2^-120); otherwise the exact row max is used.
+        float wmax_q = 0.f, wmax_k = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            wmax_q = fmaxf(wmax_q, fabsf(__bfloat162float(p.wq[4 * lane + e])));
+            wmax_k = fmaxf(wmax_k, fabsf(__bfloat162float(p.wk[4 * lane + e])));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            wmax_q = fmaxf(wmax_q, __shfl_xor_sync(0xffffffffu, wmax_q, o));
+            wmax_k = fmaxf(wmax_k, __shfl_xor_sync(0xffffffffu, wmax_k, o));
+        }
+        const float ref_fixed = 1.02f * 128.0f * wmax_q * wmax_k * fabsf(p.sl2);
+        const bool fixed = ref_fixed <= 60.0f;
         Walker w;
         w.init(p, u0);
         bool ok = true;
@@ -618,26 +636,28 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int lo = max(t + 129 - p.window, 128 - kTok * w.s);
             const int hi = t + 128;
             const uint32_t ts = tmem + lane_base + bb * 256;
-            // pass 1: row max over the visible columns (the next chunk's TMEM
-            // load is in flight while the current one is reduced)
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            {
-                uint32_t va[32], vb[32];
-                tmem_ld32(ts, va);
+            float mxs = ref_fixed;   // reference in log2 units
+            if (!fixed) {
+                // pass 1: row max over the visible columns (the next chunk's TMEM
+                // load is in flight while the current one is reduced)
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                {
+                    uint32_t va[32], vb[32];
+                    tmem_ld32(ts, va);
 #pragma unroll 1
-                for (int m = 0; m < kSpanBlocks - 1; m += 2) {
+                    for (int m = 0; m < kSpanBlocks - 1; m += 2) {
+                        tmem_wait_ld();
+                        tmem_ld32(ts + (m + 1) * 32, vb);
+                        chunk_max(va, m, lo, hi, mx4);
+                        tmem_wait_ld();
+                        tmem_ld32(ts + (m + 2) * 32, va);
+                        chunk_max(vb, m + 1, lo, hi, mx4);
+                    }
                     tmem_wait_ld();
-                    tmem_ld32(ts + (m + 1) * 32, vb);
-                    chunk_max(va, m, lo, hi, mx4);
-                    tmem_wait_ld();
-                    tmem_ld32(ts + (m + 2) * 32, va);
-                    chunk_max(vb, m + 1, lo, hi, mx4);
+                    chunk_max(va, kSpanBlocks - 1, lo, hi, mx4);
                 }
-                tmem_wait_ld();
-                chunk_max(va, kSpanBlocks - 1, lo, hi, mx4);
+                mxs = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.sl2;
             }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-            const float mxs = mx * p.sl2;
             // pass 2: P = 2^(S sl2 - max sl2) in bf16 over S's first 80 columns
             // (P of chunk m lands on S columns of chunk m/2, already consumed)
             float sum4[4] = {0.f, 0.f, 0.f, 0.f};

@@ -44,6 +44,24 @@ def test_swa_fwd_matches_oracle(name):
     assert_fwd_close(lse, lo, "lse")
 
 
+@pytest.mark.parametrize("name", ["tiny_512", "window_64_T161", "ragged_37_w16"])
+def test_swa_fwd_exact_max_path(name):
+    """One-dimension weight spikes (max|w| = 4, other weights 1) put the QK-norm
+    score bound past the range where the kernel uses it as the softmax
+    reference, so the exact row-max pass runs; the scores stay close to those
+    of unit weights."""
+    s, seed, _ = CASES[name]
+    x = attention_inputs(s, seed)
+    wq, wk = torch.ones(128), torch.ones(128)
+    wq[9], wk[100] = 4.0, 4.0
+    x["wq"], x["wk"] = wq.to(torch.bfloat16), wk.to(torch.bfloat16)
+    y, lse = run_gpu(s, x)
+    yo, lo = oracle.attn_fwd(x["q"], x["k"], x["v"], x["g"], x["wq"], x["wk"], window=s.window, gated=True,
+                             **oracle.shape_kwargs(s))
+    assert_fwd_close(y, yo, "y")
+    assert_fwd_close(lse, lo, "lse")
+
+
 def test_swa_fwd_deterministic():
     s = Shape(B=2, T=257, Hq=8, Hkv=2)
     x = attention_inputs(s, 11)
