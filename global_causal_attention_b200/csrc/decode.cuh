@@ -93,9 +93,28 @@ __device__ __forceinline__ float4 prep_head_warp(const __nv_bfloat16 *x, const _
 }
 
 // ----------------------------------------------------------------- sliding window
-__global__ void __launch_bounds__(128)
-swa_decode_kernel(const __grid_constant__ Params p)
+// One CTA per (sequence, KV head), one warp per query head.  The whole ring
+// (K and V, W rows each) is loaded by TMA into shared memory (128-byte
+// swizzle: a lane per slot reads its K row without bank conflicts) while the
+// new token's q, k and v are prepared; the new token's row is then written
+// over its slot in shared memory (and in the ring), and the attention reads
+// shared memory only.
+constexpr uint32_t kRingHalfMax = 128 * 128;   // 128 slots x 64 dims bf16: 16 KiB
+
+__device__ __forceinline__ uint32_t ring_half_bytes(int W)
 {
+    return (uint32_t)((W * 128 + 1023) / 1024 * 1024);   // halves stay 1024-byte aligned
+}
+
+constexpr uint32_t kSwaDecSmemBytes = 4 * kRingHalfMax + 16 + 1024;
+
+__global__ void __launch_bounds__(128)
+swa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
     __shared__ __align__(16) float qt[4][kD];
     __shared__ __align__(16) float ubuf[4][kD];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,23 +126,48 @@ swa_decode_kernel(const __grid_constant__ Params p)
         return;
     }
     const int W = p.W;
+    const uint32_t hs = ring_half_bytes(W);
+    const uint32_t ks = sbase, vs = sbase + 2 * hs;
+    const uint32_t bar = sbase + 4 * hs;
+    Abort ab{reinterpret_cast<volatile int *>(smem + 4 * hs + 8)};
     const int slot_new = (int)(pos % W);
     const long long cbase = ((long long)b * p.Hkv + kvh) * W;   // first row of this (b, kvh) ring
+    if (threadIdx.x == 0) {
+        *ab.flag = 0;
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(bar, 4u * (uint32_t)W * 128u);
+        for (int h = 0; h < 2; ++h) {
+            tma_load_2d(ks + h * hs, &tm_k, bar, h * 64, (int)cbase);
+            tma_load_2d(vs + h * hs, &tm_v, bar, h * 64, (int)cbase);
+        }
+    }
 
     const float4 q4 = prep_head_warp(p.q + ((long long)b * p.Hq + head) * kD, p.wq, p.R, p.eps, pos,
                                      p.theta, ubuf[warp]);
     *reinterpret_cast<float4 *>(&qt[warp][4 * lane]) = q4;
+    uint2 kbits = make_uint2(0, 0), vbits = make_uint2(0, 0);
     if (warp == 0) {
         // the new key, prepared and rounded as the cache stores it
         const float4 k4 = prep_head_warp(p.k + ((long long)b * p.Hkv + kvh) * kD, p.wk, p.R, p.eps, pos,
                                          p.theta, ubuf[0]);
-        *reinterpret_cast<uint2 *>(p.kc + (cbase + slot_new) * kD + 4 * lane) =
-            make_uint2(pack_bf16(k4.x, k4.y), pack_bf16(k4.z, k4.w));
+        kbits = make_uint2(pack_bf16(k4.x, k4.y), pack_bf16(k4.z, k4.w));
+        *reinterpret_cast<uint2 *>(p.kc + (cbase + slot_new) * kD + 4 * lane) = kbits;
     } else if (warp == 1) {
-        *reinterpret_cast<uint2 *>(p.vc + (cbase + slot_new) * kD + 4 * lane) =
-            *reinterpret_cast<const uint2 *>(p.v + ((long long)b * p.Hkv + kvh) * kD + 4 * lane);
+        vbits = *reinterpret_cast<const uint2 *>(p.v + ((long long)b * p.Hkv + kvh) * kD + 4 * lane);
+        *reinterpret_cast<uint2 *>(p.vc + (cbase + slot_new) * kD + 4 * lane) = vbits;
+    }
+    __syncthreads();   // the barrier's initialisation is visible to every waiter
+    const bool landed = warp_wait(bar, 0, ab);
+    // the new token's row over its slot (the ring load may hold either version of it)
+    if (landed && warp < 2) {
+        const uint32_t tile = warp == 0 ? ks : vs;
+        const uint32_t off = swa::chunk_off(slot_new, (4 * lane) / 8, hs) + ((4 * lane) % 8) * 2;
+        const uint2 bits = warp == 0 ? kbits : vbits;
+        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(tile + off), "r"(bits.x), "r"(bits.y) : "memory");
     }
     __syncthreads();
+    if (!landed) return;
 
     // scores: lane owns slots lane + 32 i; slot s holds position pos - ((slot_new - s) mod W)
     float sc[4];
@@ -135,11 +179,10 @@ swa_decode_kernel(const __grid_constant__ Params p)
         if (s < W) {
             const int age = (slot_new - s + W) % W;
             if (age <= pos) {
-                const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + (cbase + s) * kD);
                 float acc = 0.f;
 #pragma unroll 4
                 for (int c = 0; c < 16; ++c) {
-                    const uint4 kv = kr[c];
+                    const uint4 kv = lds128(ks + swa::chunk_off(s, c, hs));
                     const float4 qa = *reinterpret_cast<const float4 *>(&qt[warp][8 * c]);
                     const float4 qb = *reinterpret_cast<const float4 *>(&qt[warp][8 * c + 4]);
                     const float2 k0 = unpack_bf16(kv.x), k1 = unpack_bf16(kv.y), k2 = unpack_bf16(kv.z),
@@ -160,7 +203,9 @@ swa_decode_kernel(const __grid_constant__ Params p)
         l += pr[i];
     }
     l = warp_sum(l);
-    // P V: lane owns dims 4 lane .. 4 lane + 3
+    // P V: lane owns dims 4 lane .. 4 lane + 3 (half lane / 16, chunk (lane % 16) / 2, word lane % 2)
+    const uint32_t v_half = (uint32_t)(lane >> 4) * hs, v_chunk = (uint32_t)((lane & 15) >> 1),
+                   v_word = (uint32_t)(lane & 1) * 8;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i = 0; i < 4; ++i) {
 #pragma unroll 8
@@ -168,12 +213,14 @@ swa_decode_kernel(const __grid_constant__ Params p)
             const int s = 32 * i + j;
             const float ps = __shfl_sync(0xffffffffu, pr[i], j);
             if (s < W && ps != 0.f) {
-                const uint2 vv = *reinterpret_cast<const uint2 *>(p.vc + (cbase + s) * kD + 4 * lane);
-                const float2 v0 = unpack_bf16(vv.x), v1 = unpack_bf16(vv.y);
-                o[0] = fmaf(ps, v0.x, o[0]);
-                o[1] = fmaf(ps, v0.y, o[1]);
-                o[2] = fmaf(ps, v1.x, o[2]);
-                o[3] = fmaf(ps, v1.y, o[3]);
+                uint32_t v0, v1;
+                const uint32_t va = vs + v_half + (uint32_t)s * 128 + ((v_chunk ^ (uint32_t)(s & 7)) << 4) + v_word;
+                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(va));
+                const float2 f0 = unpack_bf16(v0), f1 = unpack_bf16(v1);
+                o[0] = fmaf(ps, f0.x, o[0]);
+                o[1] = fmaf(ps, f0.y, o[1]);
+                o[2] = fmaf(ps, f1.x, o[2]);
+                o[3] = fmaf(ps, f1.y, o[3]);
             }
         }
     }

@@ -82,6 +82,7 @@ int device_setup(int *num_sms)
                    set_smem(gswa::swa::swa_fwd_kernel<128>, gswa::swa::kSmemBytes) ||
                    set_smem(gswa::full::full_fwd_kernel, gswa::full::kSmemBytes) ||
                    set_smem(gswa::dec::full_decode_chunk_kernel, gswa::dec::kDecSmemBytes) ||
+                   set_smem(gswa::dec::swa_decode_kernel, gswa::dec::kSwaDecSmemBytes) ||
                    set_bwd_smem<0>() || set_bwd_smem<42>() || set_bwd_smem<64>() || set_bwd_smem<128>()) {
             d.status = GSWA_ERR_LAUNCH;
         }
@@ -603,7 +604,14 @@ int gswa_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
     p.vc = static_cast<__nv_bfloat16 *>(v_ring);
     p.pos = pos;
     p.y = static_cast<__nv_bfloat16 *>(y);
-    gswa::dec::swa_decode_kernel<<<s->B * s->Hkv, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    // ring rows as TMA coordinates (32-bit)
+    CUtensorMap tkr, tvr;
+    const long long ring_rows = (long long)s->B * s->Hkv * s->window;
+    if (ring_rows > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (encode_rows(&tkr, k_ring, ring_rows, s->window) || encode_rows(&tvr, v_ring, ring_rows, s->window))
+        return GSWA_ERR_INVALID_ARG;
+    gswa::dec::swa_decode_kernel<<<s->B * s->Hkv, 128, gswa::dec::kSwaDecSmemBytes,
+                                   static_cast<cudaStream_t>(stream)>>>(tkr, tvr, p);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
