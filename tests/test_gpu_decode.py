@@ -19,7 +19,10 @@ def _kw(R=42, base=1e4):
 
 @pytest.mark.parametrize("W,positions,R", [(128, [0, 5, 126, 127, 128, 1000, 262143], 42),
                                            (16, [0, 15, 16, 17, 300], 42),
-                                           (128, [3, 200], 0)])
+                                           (128, [3, 200], 0),
+                                           (100, [0, 99, 100, 101, 5000], 42),
+                                           (37, [36, 37, 73], 64),
+                                           (1, [0, 7], 42)])
 def test_swa_decode_matches_oracle(W, positions, R):
     B, Hq, Hkv = len(positions), 8, 2
     x = decode_inputs(B, Hq, Hkv, 128, W, seed=W + R, random_weights=True)
@@ -42,7 +45,8 @@ def test_swa_decode_matches_oracle(W, positions, R):
         assert torch.equal(vc[b, :, others], x["v_cache"][b, :, others])
 
 
-@pytest.mark.parametrize("Tmax,positions", [(9000, [0, 1, 4095, 4096, 8999]), (4096, [4095, 100])])
+@pytest.mark.parametrize("Tmax,positions", [(9000, [0, 1, 4095, 4096, 8999]), (4096, [4095, 100]),
+                                            (33, [0, 32, 31])])
 def test_full_decode_matches_oracle(Tmax, positions):
     B, Hq, Hkv = len(positions), 8, 2
     x = decode_inputs(B, Hq, Hkv, 128, Tmax, seed=Tmax, random_weights=True)
