@@ -50,7 +50,7 @@ WORKLOAD_NAMES = ["train_4k", "prefill_64k", "prefill_256k", "decode_256k"]
 LAYERS = workloads.N_LAYERS
 
 # Kernel launches of one call of each entry point.
-LAUNCHES = {"gswa_fwd": 1, "gswa_bwd": 7, "full_attn_fwd": 2, "full_attn_bwd": 7, "gswa_decode": 1,
+LAUNCHES = {"gswa_fwd": 1, "gswa_bwd": 7, "full_attn_fwd": 3, "full_attn_bwd": 7, "gswa_decode": 1,
             "full_decode": 3}
 
 # DRAM bytes (read + write) of one call, from an ncu capture of the same
