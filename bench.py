@@ -50,7 +50,7 @@ WORKLOAD_NAMES = ["train_4k", "prefill_64k", "prefill_256k", "decode_256k"]
 LAYERS = workloads.N_LAYERS
 
 # Kernel launches of one call of each entry point.
-LAUNCHES = {"gswa_fwd": 1, "gswa_bwd": 7, "full_attn_fwd": 3, "full_attn_bwd": 7, "gswa_decode": 1,
+LAUNCHES = {"gswa_fwd": 2, "gswa_bwd": 7, "full_attn_fwd": 3, "full_attn_bwd": 7, "gswa_decode": 1,
             "full_decode": 3}
 
 # DRAM bytes (read + write) of one call, from an ncu capture of the same
@@ -228,12 +228,14 @@ def build_train(s, dev, seed):
     lse_s, lse_f = f32(s.B, s.Hq, s.T), f32(s.B, s.Hq, s.T)
     g_s = (e(x["q"]), e(x["k"]), e(x["k"]), e(x["q"]), f32(s.D), f32(s.D))
     g_f = (e(x["q"]), e(x["k"]), e(x["k"]), f32(s.D), f32(s.D))
+    ws_sf = _ws(gca, gca.OP_GSWA_FWD, sh_swa, dev)
     ws_sb = _ws(gca, gca.OP_GSWA_BWD, sh_swa, dev)
     ws_ff = _ws(gca, gca.OP_FULL_FWD, sh_full, dev)
     ws_fb = _ws(gca, gca.OP_FULL_BWD, sh_full, dev)
     q, k, v, g, wq, wk, dy = (x[n] for n in ("q", "k", "v", "g", "wq", "wk", "dy"))
     calls = [
-        ("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse_s, **kw)),
+        ("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse_s, workspace=ws_sf,
+                                          **kw)),
         ("gswa_bwd", lambda: gca.gswa_bwd(q, k, v, g, wq, wk, y_s, lse_s, dy, window=s.window, workspace=ws_sb,
                                           out=g_s, **kw)),
         ("full_attn_fwd", lambda: gca.full_attn_fwd(q, k, v, wq, wk, y=y_f, lse=lse_f, workspace=ws_ff, **kw)),
@@ -250,9 +252,11 @@ def build_prefill(name, s, dev, seed):
     x = workloads.attention_inputs(s, seed, device=dev)
     kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
     sh_full = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, 0, **kw)
+    sh_swa = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, s.window, **kw)
     y_s, y_f = torch.empty_like(x["q"]), torch.empty_like(x["q"])
     lse = torch.empty(s.B, s.Hq, s.T, dtype=torch.float32, device=dev)
     ws_ff = _ws(gca, gca.OP_FULL_FWD, sh_full, dev)
+    ws_sf = _ws(gca, gca.OP_GSWA_FWD, sh_swa, dev)
     q, k, v, g, wq, wk = (x[n] for n in ("q", "k", "v", "g", "wq", "wk"))
     calls = []
     for layer in range(1, LAYERS + 1):
@@ -261,7 +265,7 @@ def build_prefill(name, s, dev, seed):
                                                                      workspace=ws_ff, **kw)))
         else:
             calls.append(("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse,
-                                                           **kw)))
+                                                           workspace=ws_sf, **kw)))
     return Step(name, s, s.B * s.T, calls, x, [y_s])
 
 

@@ -127,7 +127,7 @@ def _dev(*ts):
 
 
 def gswa_fwd(q, k, v, g, wq, wk, *, window=128, rope_dims=42, rope_base=1e4, eps=1e-6,
-             scale=None, y=None, lse=None, stream=None):
+             scale=None, y=None, lse=None, workspace=None, stream=None):
     """Gated SWA forward.  q, g [B,T,Hq,D], k, v [B,T,Hkv,D], wq, wk [D] (bf16, cuda).
     Returns (y [B,T,Hq,D] bf16, lse [B,Hq,T] f32)."""
     torch = _dev(q, k, v, g, wq, wk, y, lse)
@@ -137,8 +137,9 @@ def gswa_fwd(q, k, v, g, wq, wk, *, window=128, rope_dims=42, rope_base=1e4, eps
         y = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    ws, nb = _workspace(OP_GSWA_FWD, s, workspace, q.device)
     _check(lib().gswa_fwd(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq),
-                          _ptr(wk), _ptr(y), _ptr(lse), None, 0, _stream(stream)), "gswa_fwd")
+                          _ptr(wk), _ptr(y), _ptr(lse), _ptr(ws), nb, _stream(stream)), "gswa_fwd")
     return y, lse
 
 

@@ -184,6 +184,12 @@ size_t full_fwd_ws_keys(const gswa_shape_t *s)
     return align256((size_t)s->B * s->T * s->Hkv * s->D * 2);
 }
 
+// Workspace of the gated-SWA forward: prepared keys k~ [B, T, Hkv, D], bf16.
+size_t swa_fwd_ws(const gswa_shape_t *s)
+{
+    return align256((size_t)s->B * s->T * s->Hkv * s->D * 2);
+}
+
 size_t full_fwd_ws(const gswa_shape_t *s)
 {
     return full_fwd_ws_keys(s) + align256((size_t)s->B * s->T * s->Hq * s->D * 2);
@@ -435,8 +441,6 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
              const void *w_q, const void *w_k, void *y, float *lse, void *workspace,
              size_t workspace_bytes, void *stream)
 {
-    (void)workspace;
-    (void)workspace_bytes;
     int rc = check_common(s);
     if (rc != GSWA_OK) return rc;
     if (s->window < 1 || s->window > 128) return GSWA_ERR_UNSUPPORTED_SHAPE;
@@ -446,15 +450,24 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(y) ||
         (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
         return GSWA_ERR_MISALIGNED;
+    if (workspace == nullptr || workspace_bytes < swa_fwd_ws(s)) return GSWA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
     int num_sms = 0;
     rc = device_setup(&num_sms);
+    if (rc != GSWA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // k~ = RoPE(RMSNorm(k) w_k) once into the workspace: each key block is
+    // read by five consecutive query blocks.
+    void *kt = workspace;
+    rc = launch_qk_prep(s, s->Hkv, k, w_k, kt, 0, st, num_sms);
     if (rc != GSWA_OK) return rc;
 
     CUtensorMap tq, tk, tv, tg, ty;
     if (encode_bthd(&tq, q, s->B, s->T, s->Hq, s->D, 4, 32) ||
         encode_bthd(&tg, g, s->B, s->T, s->Hq, s->D, 4, 32) ||
         encode_bthd(&ty, y, s->B, s->T, s->Hq, s->D, 4, 32) ||
-        encode_bthd(&tk, k, s->B, s->T, s->Hkv, s->D, 1, 32) ||
+        encode_bthd(&tk, kt, s->B, s->T, s->Hkv, s->D, 1, 32) ||
         encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, 32))
         return GSWA_ERR_INVALID_ARG;
 
@@ -475,7 +488,6 @@ int gswa_fwd(const gswa_shape_t *s, const void *q, const void *k, const void *v,
     fill_theta(p.theta, s->rope_dims, s->rope_base);
 
     const long long grid = p.units < num_sms ? p.units : num_sms;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const dim3 gr((unsigned)grid), bl(gswa::swa::kThreads);
     const uint32_t sm = gswa::swa::kSmemBytes;
     switch (s->rope_dims) {
@@ -717,6 +729,7 @@ size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
 {
     if (s == nullptr || s->B < 0 || s->T < 0 || s->Hkv <= 0 || s->D <= 0) return 0;
     switch (op) {
+    case GSWA_OP_GSWA_FWD: return swa_fwd_ws(s);
     case GSWA_OP_FULL_FWD: return full_fwd_ws(s);
     case GSWA_OP_GSWA_BWD: return bwd_ws_layout(s, true).total;
     case GSWA_OP_FULL_BWD: return bwd_ws_layout(s, false).total;

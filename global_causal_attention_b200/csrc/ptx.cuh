@@ -191,6 +191,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// Prefetch one tile of a 4-D tensor map into L2 (no shared memory, no
+// completion event); coordinates outside the tensor are skipped.
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void *tmap, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int c0, int c1)
 {
     asm volatile(
@@ -395,6 +405,21 @@ __device__ __forceinline__ float tanh_approx(float x)
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// σ(x) = (1 + tanh(x/2)) / 2 of a packed bf16 pair, evaluated on f16 pairs
+// (one MUFU op per pair); returns the packed f16 pair.  A bf16 value is exact
+// in f16 over f16's normal range; outside it the f16 rounding only moves x
+// where σ is already flat (|x| > 65504 gives 0 or 1, tiny |x| gives 1/2).
+__device__ __forceinline__ uint32_t sigmoid_bf16x2_f16x2(uint32_t g)
+{
+    const uint32_t half2 = 0x38003800u;   // {0.5, 0.5} in f16
+    uint32_t h, t, s;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(__uint_as_float(g & 0xFFFF0000u)), "f"(__uint_as_float(g << 16)));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(h), "r"(half2));
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+    asm("fma.rn.f16x2 %0, %1, %2, %2;" : "=r"(s) : "r"(t), "r"(half2));
+    return s;
 }
 
 // Two floats to a packed f16 pair (`lo` in the low half), round to nearest.

@@ -5,7 +5,10 @@
 // 128, QK RMSNorm, partial RoPE; GatedSWA(h) = o_proj(A_SWA(q,k,v) ⊙ σ(g)))
 //   y_i = softmax_{i-W < j <= i}(scale <q~_i, k~_j>) V  ⊙  σ(g_i)
 // with q~, k~ the RMS-normed, partially rotated queries and keys, and the
-// natural-log normaliser lse_i of each row.
+// natural-log normaliser lse_i of each row.  The keys arrive prepared (k~,
+// written once by qk_prep: each key block serves five query blocks, and one
+// key warp per CTA preparing them in-line overloaded its scheduler); the
+// queries are prepared here, in shared memory, as their tiles land.
 //
 // Work unit: a 32-token query block of one (sequence, KV head) pair, i.e. the
 // 4 query heads of a GQA group packed as M = 128 tensor-core rows
@@ -17,12 +20,16 @@
 // ring while the window slides over it.
 //
 // Warp roles (16 warps):
-//   warp 0      TMA producer of K/V blocks (ring)
+//   warp 0      TMA producer of k~ blocks (ring); also prefetches the tiles
+//               of a later unit into L2
 //   warp 1      TMEM owner and tcgen05.mma issuer; it polls S-, PV- and
 //               Q-slot readiness independently (so none waits behind another)
 //               and also issues the TMA loads of the Q tiles (2 stages)
-//   warp 2      key prologue: RMSNorm + RoPE of each new K block, in place
-//   warp 3      idle
+//   warp 2      idle
+//   warp 3      TMA producer of V blocks (ring)
+// K and V slots have their own barriers: a K slot is handed back as soon as
+// the last QK^T that reads it completes, a V slot after the last PV, so the
+// next K block's load never waits behind a softmax.
 //   warps 4-7   query prologue: RMSNorm + RoPE of the 128 Q rows, in place
 //   warps 8-11  softmax: S (TMEM) -> P (bf16, TMEM), 1/l (TMEM), lse
 //   warps 12-15 epilogue: σ(g) into the gate tile ahead of time, then
@@ -52,6 +59,7 @@ constexpr int kRing = 6;                  // K/V ring slots
 constexpr int kSpan = kSpanBlocks * kTok; // 160
 constexpr int kThreads = 512;
 constexpr int kColInvL = 80;              // TMEM column of 1/l inside a buffer
+constexpr int kPrefetchUnits = 2;         // L2 prefetch distance of the K producer, in units
 
 // Shared-memory map (offsets from a 1024-byte-aligned base).
 constexpr uint32_t kHalfRowBytes = 128;                       // 64 bf16 per swizzled row
@@ -64,9 +72,8 @@ constexpr uint32_t kOffV = kOffK + 2 * kRingHalfBytes;        // 49152
 constexpr uint32_t kOffQ = kOffV + 2 * kRingHalfBytes;        // 98304
 constexpr uint32_t kOffG = kOffQ + 2 * kTileBytes;            // 163840
 constexpr uint32_t kOffWq = kOffG + 2 * kTileBytes;           // 229376 (f32[128])
-constexpr uint32_t kOffWk = kOffWq + 512;                     // f32[128]
-constexpr uint32_t kOffBar = kOffWk + 512;
-constexpr int kNumBars = 33;
+constexpr uint32_t kOffBar = kOffWq + 512;
+constexpr int kNumBars = 45;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kSmemUsed = kOffAbort + 4;
@@ -76,8 +83,8 @@ static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
 // Barrier indices.
 enum : int {
     BQ_FULL = 0, BQ_PREP = 2, BQ_EMPTY = 4, BG_FULL = 6, BG_EMPTY = 8,
-    BKV_FULL = 10, BKV_EMPTY = 16, BS_FULL = 22, BP_READY = 24, BO_FULL = 26,
-    BT_EMPTY = 28, BY_READY = 30, B_DRAIN = 32
+    BK_FULL = 10, BK_EMPTY = 16, BS_FULL = 22, BP_READY = 24, BO_FULL = 26,
+    BT_EMPTY = 28, BY_READY = 30, B_DRAIN = 32, BV_FULL = 33, BV_EMPTY = 39
 };
 
 struct Params {
@@ -351,9 +358,11 @@ __device__ __forceinline__ void chunk_max(const uint32_t (&v)[32], int m, int lo
 }
 
 // P = 2^(S sl2 - mxs) over one 32-column chunk m (0 outside [lo, hi]), packed
-// as bf16 pairs; accumulates the row sum in f32.
-__device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], int m, int lo, int hi, float sl2,
-                                          float mxs, float (&sum)[4], uint32_t (&pk)[16])
+// as bf16 pairs; accumulates the row sum in f32.  (One masked form for every
+// chunk: a second, unmasked copy for the interior chunks saves arithmetic but
+// costs more in instruction fetch than it saves.)
+__device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], int m, int lo, int hi, float sl2, float mxs,
+                                          float (&sum)[4], uint32_t (&pk)[16])
 {
     const int kl = lo - 32 * m, kh = hi - 32 * m;
 #pragma unroll
@@ -400,7 +409,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         *ab.flag = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(BQ_FULL + i), 1);
-            mbar_init(bar(BQ_PREP + i), 5);   // 4 query-prologue warps + key warp
+            mbar_init(bar(BQ_PREP + i), 4);   // query-prologue warps
             mbar_init(bar(BQ_EMPTY + i), 1);
             mbar_init(bar(BG_FULL + i), 1);
             mbar_init(bar(BG_EMPTY + i), 1);
@@ -411,8 +420,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(bar(BY_READY + i), 4);  // epilogue warps
         }
         for (int i = 0; i < kRing; ++i) {
-            mbar_init(bar(BKV_FULL + i), 1);
-            mbar_init(bar(BKV_EMPTY + i), 1);
+            mbar_init(bar(BK_FULL + i), 1);
+            mbar_init(bar(BK_EMPTY + i), 1);
+            mbar_init(bar(BV_FULL + i), 1);
+            mbar_init(bar(BV_EMPTY + i), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
         fence_barrier_init();
@@ -424,7 +435,6 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     if (tid < 128) {
         reinterpret_cast<float *>(smem + kOffWq)[tid] = __bfloat162float(p.wq[tid]);
-        reinterpret_cast<float *>(smem + kOffWk)[tid] = __bfloat162float(p.wk[tid]);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -435,37 +445,53 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ================================================= TMA producer: K/V ring
+    if (warp == 0 || warp == 3) {
+        // ================================================= TMA producers: K ring (warp 0), V ring (warp 3)
         if (lane == 0) {
-            uint32_t kv_fills = 0;     // parity of fills per ring slot
-            uint32_t armed = 0;        // ring slots loaded at least once
+            const bool is_k = warp == 0;
+            const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+            const uint32_t ring = sbase + (is_k ? kOffK : kOffV);
+            const int b_full = is_k ? BK_FULL : BV_FULL, b_empty = is_k ? BK_EMPTY : BV_EMPTY;
+            uint32_t fills = 0;     // parity of fills per ring slot
+            uint32_t armed = 0;     // ring slots loaded at least once
             Walker w;
             w.init(p, u0);
-            auto load_kv = [&](int kb) -> bool {
+            auto load = [&](int kb) -> bool {
                 const int slot = ring_slot(kb);
-                if (!mbar_wait(bar(BKV_EMPTY + slot), ((kv_fills >> slot) & 1u) ^ 1u, ab)) return false;
-                kv_fills ^= 1u << slot;
+                if (!mbar_wait(bar(b_empty + slot), ((fills >> slot) & 1u) ^ 1u, ab)) return false;
+                fills ^= 1u << slot;
                 armed |= 1u << slot;
-                mbar_arrive_expect_tx(bar(BKV_FULL + slot), 4 * kBlockHalfBytes);
-                for (int h = 0; h < 2; ++h) {
-                    tma_load_4d(sbase + kOffK + h * kRingHalfBytes + slot * kBlockHalfBytes, &tm_k,
-                                bar(BKV_FULL + slot), h * 64, w.kvh, kb * kTok, w.b);
-                    tma_load_4d(sbase + kOffV + h * kRingHalfBytes + slot * kBlockHalfBytes, &tm_v,
-                                bar(BKV_FULL + slot), h * 64, w.kvh, kb * kTok, w.b);
-                }
+                mbar_arrive_expect_tx(bar(b_full + slot), 2 * kBlockHalfBytes);
+                for (int h = 0; h < 2; ++h)
+                    tma_load_4d(ring + h * kRingHalfBytes + slot * kBlockHalfBytes, tm, bar(b_full + slot), h * 64,
+                                w.kvh, kb * kTok, w.b);
                 return true;
             };
+            // The K producer also prefetches into L2 the q, g, k and v tiles of
+            // the unit kPrefetchUnits ahead, so the shared-memory loads that
+            // follow wait for L2, not for HBM.
+            Walker wf;
+            wf.init(p, u0);
+            for (int i = 0; i < kPrefetchUnits && i < n; ++i) wf.next(p);
             bool ok = true;
             for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
+                if (is_k && idx + kPrefetchUnits < n) {
+                    for (int h = 0; h < 2; ++h) {
+                        tma_prefetch_l2_4d(&tm_q, h * 64, wf.kvh * 4, wf.s * kTok, wf.b);
+                        tma_prefetch_l2_4d(&tm_g, h * 64, wf.kvh * 4, wf.s * kTok, wf.b);
+                        tma_prefetch_l2_4d(&tm_k, h * 64, wf.kvh, wf.s * kTok, wf.b);
+                        tma_prefetch_l2_4d(&tm_v, h * 64, wf.kvh, wf.s * kTok, wf.b);
+                    }
+                    wf.next(p);
+                }
                 if (w.first(idx))
-                    for (int kb = w.s - 4; kb < w.s && ok; ++kb) ok = load_kv(kb);
-                if (ok) ok = load_kv(w.s);
+                    for (int kb = w.s - 4; kb < w.s && ok; ++kb) ok = load(kb);
+                if (ok) ok = load(w.s);
             }
             // Teardown: every load this thread issued must have landed before
             // the CTA's shared memory is released.
             for (int slot = 0; slot < kRing; ++slot)
-                if (armed & (1u << slot)) drain_wait(bar(BKV_FULL + slot), ((kv_fills >> slot) & 1u) ^ 1u);
+                if (armed & (1u << slot)) drain_wait(bar(b_full + slot), ((fills >> slot) & 1u) ^ 1u);
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
@@ -476,6 +502,11 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             wp.init(p, u0);
             wq.init(p, u0);
             int ns = 0, npv = 0, nq = 0;
+            // K and V loads are confirmed in their producers' order: block kkb
+            // (vkb) is the next one of unit ns's (npv's) window not yet seen
+            // landed; a ring slot's fill parity flips with every load into it
+            uint32_t k_fills = 0, v_fills = 0;
+            int kkb = ws.s - 4, vkb = wp.s - 4;
             PollWatch watch;
             while (npv < n) {
                 bool progressed = false;
@@ -494,7 +525,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (ns < n && ns <= npv + 1) {
                     const int bb = ns & 1;
                     const uint32_t ph = (ns >> 1) & 1;
-                    if (mbar_test(bar(BT_EMPTY + bb), ph ^ 1u) && mbar_test(bar(BQ_PREP + bb), ph)) {
+                    while (kkb <= ws.s) {
+                        const int ks = ring_slot(kkb);
+                        if (!mbar_test(bar(BK_FULL + ks), (k_fills >> ks) & 1u)) break;
+                        k_fills ^= 1u << ks;
+                        ++kkb;
+                        progressed = true;
+                    }
+                    if (kkb > ws.s && mbar_test(bar(BT_EMPTY + bb), ph ^ 1u) && mbar_test(bar(BQ_PREP + bb), ph)) {
                         tc_fence_after();
                         const int a = ring_slot(ws.s - 4);
                         const int n1 = (kRing - a) < kSpanBlocks ? (kRing - a) : kSpanBlocks;
@@ -514,8 +552,15 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         }
                         mma_commit(bar(BS_FULL + bb));
                         mma_commit(bar(BQ_EMPTY + bb));
+                        // K slots that no later unit of this CTA reads
+                        if (ws.last(p, ns, n)) {
+                            for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(BK_EMPTY + (a + i) % kRing));
+                        } else {
+                            mma_commit(bar(BK_EMPTY + a));
+                        }
                         ws.next(p);
                         ++ns;
+                        kkb = ws.first(ns) ? ws.s - 4 : ws.s;
                         progressed = true;
                     }
                 }
@@ -523,7 +568,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (npv < ns) {
                     const int bb = npv & 1;
                     const uint32_t ph = (npv >> 1) & 1;
-                    if (mbar_test(bar(BP_READY + bb), ph)) {
+                    while (vkb <= wp.s) {
+                        const int vs = ring_slot(vkb);
+                        if (!mbar_test(bar(BV_FULL + vs), (v_fills >> vs) & 1u)) break;
+                        v_fills ^= 1u << vs;
+                        ++vkb;
+                        progressed = true;
+                    }
+                    if (vkb > wp.s && mbar_test(bar(BP_READY + bb), ph)) {
                         tc_fence_after();
                         const int a = ring_slot(wp.s - 4);
                         const uint32_t dO = tmem + bb * 256 + 128;
@@ -535,14 +587,15 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                    idesc_pv, kk > 0);
                         }
                         mma_commit(bar(BO_FULL + bb));
-                        // Release ring slots that no later unit of this CTA reads.
+                        // V slots that no later unit of this CTA reads
                         if (wp.last(p, npv, n)) {
-                            for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(BKV_EMPTY + (a + i) % kRing));
+                            for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(BV_EMPTY + (a + i) % kRing));
                         } else {
-                            mma_commit(bar(BKV_EMPTY + a));
+                            mma_commit(bar(BV_EMPTY + a));
                         }
                         wp.next(p);
                         ++npv;
+                        vkb = wp.first(npv) ? wp.s - 4 : wp.s;
                         progressed = true;
                     }
                 }
@@ -555,32 +608,6 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int i = (nq > 2 ? nq - 2 : 0); i < nq; ++i) drain_wait(bar(BQ_FULL + (i & 1)), (i >> 1) & 1);
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ================================================= key prologue (lane = key row)
-        uint32_t kv_fills = 0;
-        const float *wk = reinterpret_cast<const float *>(smem + kOffWk);
-        // per-pair row table when it fits in registers, direct evaluation otherwise
-        using KTab = typename std::conditional<(R / 2 <= 24), RopeTab<R / 2, 1>, RopeDirect<R / 2>>::type;
-        KTab tab;
-        tab.init_rows(lane, 0, p.theta);
-        Walker w;
-        w.init(p, u0);
-        bool ok = true;
-        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
-            for (int kb = w.first(idx) ? w.s - 4 : w.s; kb <= w.s && ok; ++kb) {
-                const int slot = ring_slot(kb);
-                ok = warp_wait(bar(BKV_FULL + slot), (kv_fills >> slot) & 1u, ab);
-                kv_fills ^= 1u << slot;
-                if (ok) {
-                    tab.set_block(kb * kTok, p.theta);
-                    prep_row<R, false>(sbase + kOffK + slot * kBlockHalfBytes, kRingHalfBytes, lane, wk, p.eps,
-                                       tab);
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(BQ_PREP + (idx & 1)));
-        }
     } else if (warp >= 4 && warp < 8) {
         // ================================================= query prologue
         const int r = tid - 128;
@@ -662,22 +689,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // (P of chunk m lands on S columns of chunk m/2, already consumed)
             float sum4[4] = {0.f, 0.f, 0.f, 0.f};
             {
-                uint32_t va[32], vb[32], pk[16];
-                tmem_ld32(ts, va);
+                uint32_t va[32], pk[16];
 #pragma unroll 1
-                for (int m = 0; m < kSpanBlocks - 1; m += 2) {
+                for (int m = 0; m < kSpanBlocks; ++m) {
+                    tmem_ld32(ts + m * 32, va);
                     tmem_wait_ld();
-                    tmem_ld32(ts + (m + 1) * 32, vb);
                     chunk_exp(va, m, lo, hi, p.sl2, mxs, sum4, pk);
                     tmem_st16(ts + m * 16, pk);
-                    tmem_wait_ld();
-                    tmem_ld32(ts + (m + 2) * 32, va);
-                    chunk_exp(vb, m + 1, lo, hi, p.sl2, mxs, sum4, pk);
-                    tmem_st16(ts + (m + 1) * 16, pk);
                 }
-                tmem_wait_ld();
-                chunk_exp(va, kSpanBlocks - 1, lo, hi, p.sl2, mxs, sum4, pk);
-                tmem_st16(ts + (kSpanBlocks - 1) * 16, pk);
             }
             const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
             tmem_st1(ts + kColInvL, __float_as_uint(1.0f / sum));
@@ -722,15 +741,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int c = 0; c < 16; ++c) {
                 uint4 nxt = cur;
                 if (c + 1 < 16) nxt = lds128(ga + chunk_off(r, c + 1, kTileHalfBytes));
-                const uint32_t gu[4] = {cur.x, cur.y, cur.z, cur.w};
-                uint32_t su[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 gf = unpack_bf16(gu[e]);
-                    su[e] = pack_f16(fmaf(0.5f, tanh_approx(0.5f * gf.x), 0.5f),
-                                     fmaf(0.5f, tanh_approx(0.5f * gf.y), 0.5f));
-                }
-                sts128(ga + chunk_off(r, c, kTileHalfBytes), make_uint4(su[0], su[1], su[2], su[3]));
+                sts128(ga + chunk_off(r, c, kTileHalfBytes),
+                       make_uint4(sigmoid_bf16x2_f16x2(cur.x), sigmoid_bf16x2_f16x2(cur.y),
+                                  sigmoid_bf16x2_f16x2(cur.z), sigmoid_bf16x2_f16x2(cur.w)));
                 cur = nxt;
             }
             return true;

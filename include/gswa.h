@@ -84,7 +84,10 @@ typedef struct gswa_shape {
  *   y [B,T,Hq,D] bf16: device, written (gated output).
  *   lse [B,Hq,T] f32: device, written (natural-log softmax normaliser of each
  *     row, for the backward); may be NULL.
- *   workspace may be NULL (needs 0 bytes).
+ *   workspace: gswa_workspace_bytes(GSWA_OP_GSWA_FWD) bytes (device, 16-byte
+ *     aligned), overwritten; it receives the prepared keys k~ [B,T,Hkv,D]
+ *     (each key block is read by five consecutive query blocks, so it is
+ *     normed and rotated once).  GSWA_ERR_WORKSPACE_TOO_SMALL if smaller.
  */
 int gswa_fwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
              const void *g, const void *w_q, const void *w_k, void *y, float *lse,

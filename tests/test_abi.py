@@ -71,6 +71,16 @@ def test_null_and_misaligned_pointers(L):
     assert _call_fwd(L, s, ptr=18) == -3
 
 
+def test_fwd_workspace_holds_the_prepared_keys(L):
+    s = gca.make_shape(2, 100, 8, 2)
+    # k~ [B, T, Hkv, D] bf16, rounded up to 256 bytes
+    assert gca.workspace_bytes(gca.OP_GSWA_FWD, s) == -(-2 * 100 * 2 * 128 * 2 // 256) * 256
+    need = gca.workspace_bytes(gca.OP_GSWA_FWD, s)
+    assert L.gswa_fwd(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, None, None, 0, None) == -4
+    assert L.gswa_fwd(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, None, 16, need - 1, None) == -4
+    assert L.gswa_fwd(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, None, 24, need, None) == -3
+
+
 def test_empty_problem_is_a_no_op(L):
     s = gca.make_shape(0, 64, 4, 1)
     assert _call_fwd(L, s, ptr=0) == 0
