@@ -20,8 +20,7 @@
 // ring while the window slides over it.
 //
 // Warp roles (16 warps):
-//   warp 0      TMA producer of k~ blocks (ring); also prefetches the tiles
-//               of a later unit into L2
+//   warp 0      TMA producer of k~ blocks (ring)
 //   warp 1      TMEM owner and tcgen05.mma issuer; it polls S-, PV- and
 //               Q-slot readiness independently (so none waits behind another)
 //               and also issues the TMA loads of the Q tiles (2 stages)
@@ -59,7 +58,6 @@ constexpr int kRing = 6;                  // K/V ring slots
 constexpr int kSpan = kSpanBlocks * kTok; // 160
 constexpr int kThreads = 512;
 constexpr int kColInvL = 80;              // TMEM column of 1/l inside a buffer
-constexpr int kPrefetchUnits = 2;         // L2 prefetch distance of the K producer, in units
 
 // Shared-memory map (offsets from a 1024-byte-aligned base).
 constexpr uint32_t kHalfRowBytes = 128;                       // 64 bf16 per swizzled row
@@ -467,23 +465,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 w.kvh, kb * kTok, w.b);
                 return true;
             };
-            // The K producer also prefetches into L2 the q, g, k and v tiles of
-            // the unit kPrefetchUnits ahead, so the shared-memory loads that
-            // follow wait for L2, not for HBM.
-            Walker wf;
-            wf.init(p, u0);
-            for (int i = 0; i < kPrefetchUnits && i < n; ++i) wf.next(p);
             bool ok = true;
             for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
-                if (is_k && idx + kPrefetchUnits < n) {
-                    for (int h = 0; h < 2; ++h) {
-                        tma_prefetch_l2_4d(&tm_q, h * 64, wf.kvh * 4, wf.s * kTok, wf.b);
-                        tma_prefetch_l2_4d(&tm_g, h * 64, wf.kvh * 4, wf.s * kTok, wf.b);
-                        tma_prefetch_l2_4d(&tm_k, h * 64, wf.kvh, wf.s * kTok, wf.b);
-                        tma_prefetch_l2_4d(&tm_v, h * 64, wf.kvh, wf.s * kTok, wf.b);
-                    }
-                    wf.next(p);
-                }
                 if (w.first(idx))
                     for (int kb = w.s - 4; kb < w.s && ok; ++kb) ok = load(kb);
                 if (ok) ok = load(w.s);
