@@ -224,8 +224,9 @@ __device__ __forceinline__ void prep_row(uint32_t tile, uint32_t hs, int row, co
     constexpr int kPair = kAligned ? H / 8 : 0;  // aligned: chunk c pairs with chunk c + kPair
     const float4 *w4 = reinterpret_cast<const float4 *>(w);
     const int lane = threadIdx.x & 31;
-    // pass 1: mean square of the raw row (eight independent accumulators)
-    float ss[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // pass 1: mean square of the raw row (eight independent accumulators,
+    // updated in pairs by f32x2 FMAs)
+    uint64_t ss2[4] = {0, 0, 0, 0};
 #pragma unroll 4
     for (int c = 0; c < 16; ++c) {
         const uint4 v = lds128(tile + chunk_off(row, c, hs));
@@ -233,22 +234,31 @@ __device__ __forceinline__ void prep_row(uint32_t tile, uint32_t hs, int row, co
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = unpack_bf16(u4[e]);
-            ss[2 * e] = fmaf(f.x, f.x, ss[2 * e]);
-            ss[2 * e + 1] = fmaf(f.y, f.y, ss[2 * e + 1]);
+            const uint64_t x2 = f2_pack(f.x, f.y);
+            ss2[e] = f2_fma(x2, x2, ss2[e]);
         }
+    }
+    float ss[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 t = f2_unpack(ss2[e]);
+        ss[2 * e] = t.x;
+        ss[2 * e + 1] = t.y;
     }
     const float r = rsqrtf(((ss[0] + ss[1]) + (ss[2] + ss[3]) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) *
                                (1.0f / kD) + eps);
-    // scaled values of one chunk
+    const uint64_t r2 = f2_pack(r, r);
+    // scaled values x (r w) of one chunk, two dims per instruction
     auto scale8 = [&](const uint4 v, int c, float (&u)[8]) {
         const float4 wa = w4[2 * c], wb = w4[2 * c + 1];
-        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        const uint64_t w2[4] = {f2_pack(wa.x, wa.y), f2_pack(wa.z, wa.w), f2_pack(wb.x, wb.y), f2_pack(wb.z, wb.w)};
         const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = unpack_bf16(u4[e]);
-            u[2 * e] = f.x * (r * wv[2 * e]);
-            u[2 * e + 1] = f.y * (r * wv[2 * e + 1]);
+            const float2 y = f2_unpack(f2_mul(f2_pack(f.x, f.y), f2_mul(r2, w2[e])));
+            u[2 * e] = y.x;
+            u[2 * e + 1] = y.y;
         }
     };
     auto pack8 = [](const float *u) {
@@ -360,16 +370,18 @@ __device__ __forceinline__ void chunk_max(const uint32_t (&v)[32], int m, int lo
 // chunk: a second, unmasked copy for the interior chunks saves arithmetic but
 // costs more in instruction fetch than it saves.)
 __device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], int m, int lo, int hi, float sl2, float mxs,
-                                          float (&sum)[4], uint32_t (&pk)[16])
+                                          uint64_t (&sum2)[4], uint32_t (&pk)[16])
 {
     const int kl = lo - 32 * m, kh = hi - 32 * m;
+    const uint64_t sl2_2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mxs, -mxs);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(v[e]), sl2, -mxs));
-        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -mxs));
+        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sl2_2, nm2));
+        float p0 = ex2(x.x);
+        float p1 = ex2(x.y);
         p0 = (e >= kl && e <= kh) ? p0 : 0.f;
         p1 = (e + 1 >= kl && e + 1 <= kh) ? p1 : 0.f;
-        sum[(e >> 1) & 3] += p0 + p1;
+        sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(p0, p1));
         pk[e >> 1] = pack_bf16(p0, p1);
     }
 }
@@ -670,18 +682,19 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // pass 2: P = 2^(S sl2 - max sl2) in bf16 over S's first 80 columns
             // (P of chunk m lands on S columns of chunk m/2, already consumed)
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            uint64_t sum2[4] = {0, 0, 0, 0};   // eight partial sums, in pairs
             {
                 uint32_t va[32], pk[16];
 #pragma unroll 1
                 for (int m = 0; m < kSpanBlocks; ++m) {
                     tmem_ld32(ts + m * 32, va);
                     tmem_wait_ld();
-                    chunk_exp(va, m, lo, hi, p.sl2, mxs, sum4, pk);
+                    chunk_exp(va, m, lo, hi, p.sl2, mxs, sum2, pk);
                     tmem_st16(ts + m * 16, pk);
                 }
             }
-            const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            const float2 s01 = f2_unpack(f2_add(sum2[0], sum2[1])), s23 = f2_unpack(f2_add(sum2[2], sum2[3]));
+            const float sum = (s01.x + s01.y) + (s23.x + s23.y);
             tmem_st1(ts + kColInvL, __float_as_uint(1.0f / sum));
             tmem_wait_st();
             const int i = w.s * kTok + t;
@@ -742,6 +755,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t tb = tmem + lane_base + bb * 256;
             const uint32_t gaddr = sbase + kOffG + bb * kTileBytes;
             const float inv = __uint_as_float(tmem_ld1(tb + kColInvL));
+            const uint64_t inv2 = f2_pack(inv, inv);
             auto load_s = [&](int m, uint4 (&sv)[4]) {
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) sv[c4] = lds128(gaddr + chunk_off(r, m * 4 + c4, kTileHalfBytes));
@@ -755,8 +769,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 sg = unpack_f16(su[e]);
-                        yu[e] = pack_bf16(__uint_as_float(o[c4 * 8 + 2 * e]) * inv * sg.x,
-                                          __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv * sg.y);
+                        const uint64_t o2 = f2_pack(__uint_as_float(o[c4 * 8 + 2 * e]), __uint_as_float(o[c4 * 8 + 2 * e + 1]));
+                        const float2 y = f2_unpack(f2_mul(f2_mul(o2, inv2), f2_pack(sg.x, sg.y)));
+                        yu[e] = pack_bf16(y.x, y.y);
                     }
                     sts128(gaddr + chunk_off(r, m * 4 + c4, kTileHalfBytes), make_uint4(yu[0], yu[1], yu[2], yu[3]));
                 }
