@@ -586,6 +586,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int i = x.qb * 32 + (r >> 2);
             const float2 rec = p.ld[(((long long)x.b * p.Hkv + x.kvh) * p.Tp + x.qb * 32) * 4 + r];
             const float lse2 = rec.x, Dv = rec.y;
+            const uint64_t sl2_2 = f2_pack(p.sl2, p.sl2), nlse2 = f2_pack(-lse2, -lse2), nD2 = f2_pack(-Dv, -Dv);
             for (int j = 0; j < x.n && ok; ++j, ++g) {
                 const int bb = g % kNBuf;
                 ok = warp_wait(bar(C::BS_FULL + bb), (g / kNBuf) & 1, ab);
@@ -603,13 +604,17 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
+                        // two columns per f32x2 instruction (same per-lane rounding)
                         const int col = 32 * c + e;
-                        float p0 = ex2(fmaf(__uint_as_float(s[e]), p.sl2, -lse2));
-                        float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), p.sl2, -lse2));
+                        const float2 x = f2_unpack(
+                            f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2_2, nlse2));
+                        float p0 = ex2(x.x);
+                        float p1 = ex2(x.y);
                         p0 = (col >= lo && col <= hi) ? p0 : 0.f;
                         p1 = (col + 1 >= lo && col + 1 <= hi) ? p1 : 0.f;
-                        pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(d[e]) - Dv),
-                                               p1 * (__uint_as_float(d[e + 1]) - Dv));
+                        const uint64_t dd = f2_add(f2_pack(__uint_as_float(d[e]), __uint_as_float(d[e + 1])), nD2);
+                        const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), dd));
+                        pk[e >> 1] = pack_bf16(ds.x, ds.y);
                     }
                     tmem_st16(ts + 16 * c, pk);
                 }
