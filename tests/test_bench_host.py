@@ -1,0 +1,81 @@
+"""Host-side arithmetic of bench.py (no GPU): the algorithmic work every
+roofline fraction divides by, checked against closed forms written out from
+the layouts (bf16 q, k, v, g, y, dy; f32 lse) and against brute-force pair
+counts."""
+import pytest
+
+import bench
+import workloads
+from workloads import WORKLOADS, Shape
+
+
+def brute_pairs(T, W=None):
+    """(query, key) pairs with j <= i, and i - j < W for a window W."""
+    return sum(1 for i in range(T) for j in range(i + 1) if W is None or i - j < W)
+
+
+@pytest.mark.parametrize("T,W", [(1, 1), (5, 1), (7, 3), (60, 128), (128, 128), (129, 128), (300, 128)])
+def test_pair_counts_match_brute_force(T, W):
+    assert bench.swa_pairs(T, W) == brute_pairs(T, W)
+    assert bench.causal_pairs(T) == brute_pairs(T)
+
+
+def test_gswa_fwd_bytes_per_token():
+    # q and g read, y written: 3 x 32 heads x 128 x 2 B; k and v read: 2 x 8 x 128 x 2 B;
+    # lse written: 32 x 4 B  ->  24,576 + 4,096 + 128 = 28,800 B per token
+    s = WORKLOADS["train_4k"]
+    assert bench.algorithmic_work("gswa_fwd", s) == ("hbm", 8 * 4096 * 28_800, "GB/s")
+    assert 8 * 4096 * 28_800 == 943_718_400
+
+
+def test_gswa_bwd_bytes_per_token():
+    # read q, g, y, dy (4 x 8,192) and k, v (2 x 2,048) and lse (128);
+    # write dq, dg (2 x 8,192) and dk, dv (2 x 2,048)  ->  57,472 B per token
+    s = WORKLOADS["train_4k"]
+    assert bench.algorithmic_work("gswa_bwd", s) == ("hbm", 8 * 4096 * 57_472, "GB/s")
+
+
+def test_full_attention_flops():
+    # forward: QK^T and PV, 2 x 2 x D flops per visible (causal) pair and head
+    s = WORKLOADS["train_4k"]
+    fwd = 4 * 128 * 8 * 32 * (4096 * 4097 // 2)
+    assert fwd == 1_099_780_063_232
+    assert bench.algorithmic_work("full_attn_fwd", s) == ("tensor", fwd, "TFLOP/s")
+    # backward: dV, dP, dQ, dK (recomputation of S and dP not counted)
+    assert bench.algorithmic_work("full_attn_bwd", s) == ("tensor", 2 * fwd, "TFLOP/s")
+
+
+def test_decode_bytes():
+    d = workloads.DECODE_256K
+    s = Shape(B=d["B"], T=1, Hq=d["Hq"], Hkv=d["Hkv"], window=d["window"], rope_base=d["rope_base"])
+    pos = d["pos"]
+    # linear cache: K and V rows 0..pos of 8 heads, plus new q, y (32 heads) and k, v (8 heads)
+    per_seq = 2 * 8 * (pos + 1) * 128 * 2 + 2 * 32 * 128 * 2 + 2 * 8 * 128 * 2
+    assert bench.algorithmic_work("full_decode", s, pos) == ("hbm", 32 * per_seq, "GB/s")
+    assert 32 * per_seq == 34_360_393_728
+    # ring: the min(pos + 1, 128) visible slots, plus new q, g, y and k, v
+    for p, vis in ((5, 6), (127, 128), (pos, 128)):
+        ring = 32 * (2 * 8 * vis * 128 * 2 + 3 * 32 * 128 * 2 + 2 * 8 * 128 * 2)
+        assert bench.algorithmic_work("gswa_decode", s, p) == ("hbm", ring, "GB/s")
+
+
+def test_op_table_fraction():
+    """achieved = algorithmic amount / time per call; frac = achieved / peak."""
+    s = WORKLOADS["train_4k"]
+    step = bench.Step("t", s, s.B * s.T, [("gswa_fwd", None), ("full_attn_fwd", None), ("gswa_fwd", None)], {}, [])
+    K = 4
+    op_ms = {"gswa_fwd": 2 * K * 0.5, "full_attn_fwd": K * 2.0}   # 0.5 ms and 2.0 ms per call
+    pk = dict(hbm_gbs=6536.7, bf16_tflops_sustained=1387.5)
+    t = bench.op_table(step, op_ms, K, pk)
+    assert t["gswa_fwd"]["calls_per_step"] == 2
+    assert t["gswa_fwd"]["achieved"] == pytest.approx(943_718_400 / 0.5e-3 / 1e9)
+    assert t["gswa_fwd"]["frac"] == pytest.approx(943_718_400 / 0.5e-3 / 1e9 / 6536.7)
+    assert t["full_attn_fwd"]["achieved"] == pytest.approx(1_099_780_063_232 / 2.0e-3 / 1e12)
+    assert t["full_attn_fwd"]["frac"] == pytest.approx(1_099_780_063_232 / 2.0e-3 / 1e12 / 1387.5)
+    assert step.launches() == 2 * bench.LAUNCHES["gswa_fwd"] + bench.LAUNCHES["full_attn_fwd"]
+
+
+def test_every_entry_point_has_a_launch_count():
+    ops = {"gswa_fwd", "gswa_bwd", "full_attn_fwd", "full_attn_bwd", "gswa_decode", "full_decode"}
+    assert set(bench.LAUNCHES) == ops
+    assert all(n >= 1 for n in bench.LAUNCHES.values())
