@@ -15,11 +15,13 @@
 // Kernels:
 //   bwd_prep     per row: D and lse log2 e into a row-ordered record, dA and
 //                dg (gated only)
-//   bwd_dq       query-stationary (M = 128 rows = 4 heads x 32 tokens): per key
-//                tile S = Q~K~^T and dP = dA V^T into TMEM; P from the
-//                forward's lse; dS (bf16, over S); dQ~ += dS K~ in TMEM;
-//                epilogue: RoPE^T and the RMSNorm backward against the raw q,
-//                per-warp dw_q partials
+//   bwd_dq_swa / bwd_dq_full
+//                query-stationary (M = 128 rows = 4 heads x 32 tokens): S =
+//                Q~K~^T and dP = dA V^T into TMEM (sliding window: the unit's
+//                160-key span from K~/V rings kept across consecutive units;
+//                full: 64-key tiles); P from the forward's lse; dS (bf16);
+//                dQ~ += dS K~ in TMEM; epilogue: RoPE^T and the RMSNorm
+//                backward against the raw q, per-warp dw_q partials
 //   bwd_dkdv     key-stationary (M = 128 keys of one kv head): per 64-row
 //                query chunk (16 tokens x 4 heads) S^T = K~Q~^T and
 //                dP^T = V dA^T; P^T and dS^T (bf16, over S^T and dP^T);
@@ -427,14 +429,84 @@ struct DqWalk {
     }
 };
 
-template <int R, bool kSwa>
-__global__ void __launch_bounds__(kThreads, 1)
-bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
-              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-              const __grid_constant__ Params p)
+// ====================================================== dq kernel, sliding window
+// Query-stationary: unit = 32 query tokens x 4 heads (M = 128 rows) of one
+// (sequence, KV head); its keys are the 160 keys [32 s - 128, 32 s + 32), five
+// 32-key blocks.  Persistent CTAs walk a contiguous range of units, strip by
+// strip, and keep the K~ and V blocks in six-slot rings (each block is loaded
+// once per CTA and serves the five units whose window covers it); Q~ and dA
+// tiles have two slots each.  S = Q~K~^T and dP = dA V^T (N = 160, split where
+// the window wraps the ring) go to one TMEM buffer; dS = P (dP - D) is written
+// as bf16 over S; dQ~ += dS K~ is a TMEM-A MMA over the K~ ring.
+struct DqSwaCfg {
+    static constexpr int kTok = 32, kSpanBlocks = 5, kRing = 6, kSpan = kSpanBlocks * kTok;
+    static constexpr uint32_t kBlockHalf = kTok * kHalfRowBytes;    // 4 KiB: 32 keys x 64 dims
+    static constexpr uint32_t kRingHalf = kRing * kBlockHalf;       // 24 KiB
+    static constexpr uint32_t kTileHalf = 128 * kHalfRowBytes;      // 16 KiB: 128 rows x 64 dims
+    static constexpr uint32_t kTile = 2 * kTileHalf;                // 32 KiB
+    static constexpr uint32_t kOffK = 0;
+    static constexpr uint32_t kOffV = kOffK + 2 * kRingHalf;        // rings: 48 KiB each
+    static constexpr uint32_t kOffQ = kOffV + 2 * kRingHalf;        // Q~: 2 slots
+    static constexpr uint32_t kOffA = kOffQ + 2 * kTile;            // dA: 2 slots
+    static constexpr uint32_t kOffW = kOffA + 2 * kTile;            // f32[128]
+    static constexpr uint32_t kOffBar = kOffW + 512;
+    static constexpr int kNumBars = 34;
+    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    // TMEM columns: S (dS as bf16 over its first 80), dP, dQ~
+    static constexpr uint32_t kColS = 0, kColDP = kSpan, kColDQ = 2 * kSpan;
+    static_assert(kColDQ + 128 <= 512, "TMEM budget");
+    static constexpr int BQ_FULL = 0, BQ_EMPTY = 2, BK_FULL = 4, BK_EMPTY = BK_FULL + kRing,
+                         BV_FULL = BK_EMPTY + kRing, BV_EMPTY = BV_FULL + kRing, BS_FULL = BV_EMPTY + kRing,
+                         BS_FREE = BS_FULL + 1, BDS_READY = BS_FREE + 1, BACC_FULL = BDS_READY + 1,
+                         BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1;
+    static_assert(B_DRAIN < kNumBars, "barrier count");
+};
+
+// Walks units [u0, u1) of a CTA in order: (sequence b, kv head, query block s).
+struct SwaWalk {
+    int b, kvh, s;
+    __device__ __forceinline__ void init(const Params &p, long long u0)
+    {
+        const long long strip = u0 / p.nq;
+        s = (int)(u0 - strip * p.nq);
+        b = (int)(strip / p.Hkv);
+        kvh = (int)(strip - (long long)b * p.Hkv);
+    }
+    __device__ __forceinline__ void next(const Params &p)
+    {
+        if (++s == p.nq) {
+            s = 0;
+            if (++kvh == p.Hkv) {
+                kvh = 0;
+                ++b;
+            }
+        }
+    }
+    // first unit of the CTA or of a strip: its window's older blocks are not in the ring yet
+    __device__ __forceinline__ bool first(int idx) const { return idx == 0 || s == 0; }
+    // last unit of the CTA or of a strip: no later unit reads its window's blocks
+    __device__ __forceinline__ bool last(const Params &p, int idx, int n) const
+    {
+        return idx == n - 1 || s == p.nq - 1;
+    }
+};
+
+__device__ __forceinline__ int dq_ring_slot(int kb)
 {
-    using C = DqCfg<kSwa>;
-    constexpr int kN = C::kN, kNBuf = C::kNBuf, kStages = C::kStages;
+    return ((kb % DqSwaCfg::kRing) + DqSwaCfg::kRing) % DqSwaCfg::kRing;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ Params p)
+{
+    using C = DqSwaCfg;
+    constexpr int kRing = C::kRing, kSpanBlocks = C::kSpanBlocks, kTok = C::kTok;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -442,21 +514,25 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
     Abort ab{reinterpret_cast<volatile int *>(smem + C::kOffAbort)};
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * (uint32_t)i; };
-    const int nunits = snake_count(p.units);
+    const long long u0 = (long long)blockIdx.x * p.units / gridDim.x;
+    const long long u1 = (long long)(blockIdx.x + 1) * p.units / gridDim.x;
+    const int n = (int)(u1 - u0);
 
     if (tid == 0) {
         *ab.flag = 0;
-        mbar_init(bar(C::BQ_FULL), 1);
-        mbar_init(bar(C::BQ_EMPTY), 1);
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(bar(C::BKV_FULL + i), 1);
-            mbar_init(bar(C::BKV_EMPTY + i), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::BQ_FULL + i), 1);
+            mbar_init(bar(C::BQ_EMPTY + i), 1);
         }
-        for (int i = 0; i < kNBuf; ++i) {
-            mbar_init(bar(C::BS_FULL + i), 1);
-            mbar_init(bar(C::BDS_READY + i), 4);
-            mbar_init(bar(C::BS_FREE + i), 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(bar(C::BK_FULL + i), 1);
+            mbar_init(bar(C::BK_EMPTY + i), 1);
+            mbar_init(bar(C::BV_FULL + i), 1);
+            mbar_init(bar(C::BV_EMPTY + i), 1);
         }
+        mbar_init(bar(C::BS_FULL), 1);
+        mbar_init(bar(C::BS_FREE), 1);
+        mbar_init(bar(C::BDS_READY), 4);
         mbar_init(bar(C::BACC_FULL), 1);
         mbar_init(bar(C::BACC_FREE), 4);
         mbar_init(bar(C::B_DRAIN), 1);
@@ -476,93 +552,147 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ================================================= TMA producer
+    if (warp == 0 || warp == 2) {
+        // ================================================= ring producers: K~ (warp 0), V (warp 2)
         if (lane == 0) {
-            int g = 0, k = 0;
-            QUnit x;
+            const bool is_k = warp == 0;
+            const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+            const uint32_t ring = sbase + (is_k ? C::kOffK : C::kOffV);
+            const int b_full = is_k ? C::BK_FULL : C::BV_FULL, b_empty = is_k ? C::BK_EMPTY : C::BV_EMPTY;
+            uint32_t fills = 0, armed = 0;   // fill parity per slot; slots loaded at least once
+            SwaWalk w;
+            w.init(p, u0);
+            auto load = [&](int kb) -> bool {
+                const int slot = dq_ring_slot(kb);
+                if (!mbar_wait(bar(b_empty + slot), ((fills >> slot) & 1u) ^ 1u, ab)) return false;
+                fills ^= 1u << slot;
+                armed |= 1u << slot;
+                mbar_arrive_expect_tx(bar(b_full + slot), 2 * C::kBlockHalf);
+                for (int h = 0; h < 2; ++h)
+                    tma_load_4d(ring + h * C::kRingHalf + slot * C::kBlockHalf, tm, bar(b_full + slot), h * 64,
+                                w.kvh, kb * kTok, w.b);
+                return true;
+            };
             bool ok = true;
-            for (; k < nunits && ok; ++k) {
-                dq_unit_at<kSwa>(p, k, x);
-                ok = mbar_wait(bar(C::BQ_EMPTY), (k & 1) ^ 1u, ab);
+            for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
+                if (w.first(idx))
+                    for (int kb = w.s - 4; kb < w.s && ok; ++kb) ok = load(kb);
+                if (ok) ok = load(w.s);
+            }
+            for (int slot = 0; slot < kRing; ++slot)
+                if (armed & (1u << slot)) drain_wait(bar(b_full + slot), ((fills >> slot) & 1u) ^ 1u);
+        }
+    } else if (warp == 3) {
+        // ================================================= Q~ and dA tiles (two slots)
+        if (lane == 0) {
+            SwaWalk w;
+            w.init(p, u0);
+            int idx = 0;
+            bool ok = true;
+            for (; idx < n && ok; ++idx, w.next(p)) {
+                const int j = idx & 1;
+                ok = mbar_wait(bar(C::BQ_EMPTY + j), ((idx >> 1) & 1) ^ 1u, ab);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar(C::BQ_FULL), 2 * C::kQTile);
+                mbar_arrive_expect_tx(bar(C::BQ_FULL + j), 2 * C::kTile);
                 for (int h = 0; h < 2; ++h) {
-                    tma_load_4d(sbase + C::kOffQ + h * C::kQHalf, &tm_q, bar(C::BQ_FULL), h * 64, x.kvh * 4,
-                                x.qb * 32, x.b);
-                    tma_load_4d(sbase + C::kOffA + h * C::kQHalf, &tm_a, bar(C::BQ_FULL), h * 64, x.kvh * 4,
-                                x.qb * 32, x.b);
-                }
-                for (int j = 0; j < x.n && ok; ++j, ++g) {
-                    const int st = g % kStages;
-                    ok = mbar_wait(bar(C::BKV_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(bar(C::BKV_FULL + st), 2 * C::kKTile);
-                    const int key0 = dq_tile_key0<kSwa>(x, j);
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_4d(sbase + C::kOffK + st * C::kKTile + h * C::kKHalf, &tm_k,
-                                    bar(C::BKV_FULL + st), h * 64, x.kvh, key0, x.b);
-                        tma_load_4d(sbase + C::kOffV + st * C::kKTile + h * C::kKHalf, &tm_v,
-                                    bar(C::BKV_FULL + st), h * 64, x.kvh, key0, x.b);
-                    }
+                    tma_load_4d(sbase + C::kOffQ + j * C::kTile + h * C::kTileHalf, &tm_q, bar(C::BQ_FULL + j),
+                                h * 64, w.kvh * 4, w.s * kTok, w.b);
+                    tma_load_4d(sbase + C::kOffA + j * C::kTile + h * C::kTileHalf, &tm_a, bar(C::BQ_FULL + j),
+                                h * 64, w.kvh * 4, w.s * kTok, w.b);
                 }
             }
-            // no copy may still be landing when the CTA exits
-            for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
-                drain_wait(bar(C::BKV_FULL + i % kStages), (i / kStages) & 1);
-            if (k > 0) drain_wait(bar(C::BQ_FULL), (k - 1) & 1);
+            for (int i = (idx > 2 ? idx - 2 : 0); i < idx; ++i) drain_wait(bar(C::BQ_FULL + (i & 1)), (i >> 1) & 1);
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(128, kN, 0, 0);
             const uint32_t idesc_dq = idesc_bf16_f32(128, 128, 0, 1);
-            DqWalk<kSwa> ws, wd;
-            ws.init(p);
-            wd.init(p);
+            SwaWalk ws, wd;
+            ws.init(p, u0);
+            wd.init(p, u0);
             int ns = 0, nd = 0;
+            // K~ and V loads are confirmed in their producers' order: block kkb
+            // (vkb) is the next one of unit ns's window not yet seen landed
+            uint32_t k_fills = 0, v_fills = 0;
+            int kkb = ws.s - 4, vkb = ws.s - 4;
             PollWatch watch;
-            while (wd.valid) {
+            while (nd < n) {
                 bool progressed = false;
-                if (ws.valid && ns < nd + kNBuf && mbar_test(bar(C::BQ_FULL), ws.k & 1) &&
-                    mbar_test(bar(C::BKV_FULL + ns % kStages), (ns / kStages) & 1) &&
-                    mbar_test(bar(C::BS_FREE + ns % kNBuf), ((ns / kNBuf) & 1) ^ 1u)) {
-                    tc_fence_after();
-                    const uint32_t dS = tmem + (ns % kNBuf) * 2 * kN;
-                    const uint32_t ks = sbase + C::kOffK + (ns % kStages) * C::kKTile;
-                    const uint32_t vs = sbase + C::kOffV + (ns % kStages) * C::kKTile;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t oq = (kk >> 2) * C::kQHalf + (kk & 3) * 32;
-                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
-                        mma_ss(dS, smem_desc_sw128(sbase + C::kOffQ + oq, 16, 1024),
-                               smem_desc_sw128(ks + ok_, 16, 1024), idesc_s, kk > 0);
+                // S(ns) = Q~ K~^T and dP(ns) = dA V^T, once dQ(ns - 1) has read dS(ns - 1)
+                if (ns < n && ns == nd) {
+                    while (kkb <= ws.s) {
+                        const int ks = dq_ring_slot(kkb);
+                        if (!mbar_test(bar(C::BK_FULL + ks), (k_fills >> ks) & 1u)) break;
+                        k_fills ^= 1u << ks;
+                        ++kkb;
+                        progressed = true;
                     }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t oq = (kk >> 2) * C::kQHalf + (kk & 3) * 32;
-                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
-                        mma_ss(dS + kN, smem_desc_sw128(sbase + C::kOffA + oq, 16, 1024),
-                               smem_desc_sw128(vs + ok_, 16, 1024), idesc_s, kk > 0);
+                    while (vkb <= ws.s) {
+                        const int vs = dq_ring_slot(vkb);
+                        if (!mbar_test(bar(C::BV_FULL + vs), (v_fills >> vs) & 1u)) break;
+                        v_fills ^= 1u << vs;
+                        ++vkb;
+                        progressed = true;
                     }
-                    mma_commit(bar(C::BS_FULL + ns % kNBuf));
-                    if (ws.last()) mma_commit(bar(C::BQ_EMPTY));
-                    ws.next(p);
-                    ++ns;
-                    progressed = true;
+                    const int j = ns & 1;
+                    if (kkb > ws.s && vkb > ws.s && mbar_test(bar(C::BQ_FULL + j), (ns >> 1) & 1) &&
+                        mbar_test(bar(C::BS_FREE), (ns & 1) ^ 1u)) {
+                        tc_fence_after();
+                        const int a = dq_ring_slot(ws.s - 4);
+                        const int n1 = (kRing - a) < kSpanBlocks ? (kRing - a) : kSpanBlocks;
+                        const int n2 = kSpanBlocks - n1;
+                        const uint32_t id1 = idesc_bf16_f32(128, n1 * kTok, 0, 0);
+                        const uint32_t id2 = idesc_bf16_f32(128, n2 > 0 ? n2 * kTok : 32, 0, 0);
+#pragma unroll
+                        for (int op = 0; op < 2; ++op) {
+                            // op 0: S from Q~ and the K~ ring; op 1: dP from dA and the V ring
+                            const uint32_t dst = tmem + (op == 0 ? C::kColS : C::kColDP);
+                            const uint32_t at = sbase + (op == 0 ? C::kOffQ : C::kOffA) + j * C::kTile;
+                            const uint32_t rg = sbase + (op == 0 ? C::kOffK : C::kOffV);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t h = kk >> 2, ko = (kk & 3) * 32;
+                                const uint64_t ad = smem_desc_sw128(at + h * C::kTileHalf + ko, 16, 1024);
+                                const uint32_t rbase = rg + h * C::kRingHalf + ko;
+                                mma_ss(dst, ad, smem_desc_sw128(rbase + a * C::kBlockHalf, 16, 1024), id1, kk > 0);
+                                if (n2 > 0)
+                                    mma_ss(dst + n1 * kTok, ad, smem_desc_sw128(rbase, 16, 1024), id2, kk > 0);
+                            }
+                        }
+                        mma_commit(bar(C::BS_FULL));
+                        mma_commit(bar(C::BQ_EMPTY + j));
+                        // V slots that no later unit of this CTA reads (dP was their last use)
+                        if (ws.last(p, ns, n)) {
+                            for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(C::BV_EMPTY + (a + i) % kRing));
+                        } else {
+                            mma_commit(bar(C::BV_EMPTY + a));
+                        }
+                        ws.next(p);
+                        ++ns;
+                        kkb = vkb = ws.first(ns) ? ws.s - 4 : ws.s;
+                        progressed = true;
+                    }
                 }
-                if (nd < ns && mbar_test(bar(C::BDS_READY + nd % kNBuf), (nd / kNBuf) & 1) &&
-                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
+                // dQ~(nd) = dS K~ over the same window, once the epilogue has read dQ~(nd - 1)
+                if (nd < ns && mbar_test(bar(C::BDS_READY), nd & 1) &&
+                    mbar_test(bar(C::BACC_FREE), (nd & 1) ^ 1u)) {
                     tc_fence_after();
-                    const uint32_t ks = sbase + C::kOffK + (nd % kStages) * C::kKTile;
-                    const uint32_t da = tmem + (nd % kNBuf) * 2 * kN;
+                    const int a = dq_ring_slot(wd.s - 4);
 #pragma unroll
-                    for (int kk = 0; kk < kN / 16; ++kk)
-                        mma_ts(tmem + C::kColDQ, da + kk * 8, smem_desc_sw128(ks + kk * 16 * 128, C::kKHalf, 1024),
-                               idesc_dq, (wd.j > 0 || kk > 0));
-                    mma_commit(bar(C::BKV_EMPTY + nd % kStages));
-                    mma_commit(bar(C::BS_FREE + nd % kNBuf));
-                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
+                    for (int kk = 0; kk < C::kSpan / 16; ++kk) {
+                        const int slot = (a + (kk >> 1)) % kRing;
+                        const uint32_t kaddr = sbase + C::kOffK + slot * C::kBlockHalf + (kk & 1) * 16 * kHalfRowBytes;
+                        mma_ts(tmem + C::kColDQ, tmem + C::kColS + kk * 8, smem_desc_sw128(kaddr, C::kRingHalf, 1024),
+                               idesc_dq, kk > 0);
+                    }
+                    mma_commit(bar(C::BS_FREE));
+                    mma_commit(bar(C::BACC_FULL));
+                    // K~ slots that no later unit of this CTA reads
+                    if (wd.last(p, nd, n)) {
+                        for (int i = 0; i < kSpanBlocks; ++i) mma_commit(bar(C::BK_EMPTY + (a + i) % kRing));
+                    } else {
+                        mma_commit(bar(C::BK_EMPTY + a));
+                    }
                     wd.next(p);
                     ++nd;
                     progressed = true;
@@ -574,55 +704,52 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
-        // ================================================= dS = P (dP - D)
+        // ================================================= dS = P (dP - D), bf16 over S
         const int r = tid - 128;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const int W = kSwa ? p.window : 0;
+        const int W = p.window;
+        const uint64_t sl2_2 = f2_pack(p.sl2, p.sl2);
+        SwaWalk w;
+        w.init(p, u0);
         bool ok = true;
-        int g = 0;
-        QUnit x;
-        for (int k = 0; k < nunits && ok; ++k) {
-            dq_unit_at<kSwa>(p, k, x);
-            const int i = x.qb * 32 + (r >> 2);
-            const float2 rec = p.ld[(((long long)x.b * p.Hkv + x.kvh) * p.Tp + x.qb * 32) * 4 + r];
-            const float lse2 = rec.x, Dv = rec.y;
-            const uint64_t sl2_2 = f2_pack(p.sl2, p.sl2), nlse2 = f2_pack(-lse2, -lse2), nD2 = f2_pack(-Dv, -Dv);
-            for (int j = 0; j < x.n && ok; ++j, ++g) {
-                const int bb = g % kNBuf;
-                ok = warp_wait(bar(C::BS_FULL + bb), (g / kNBuf) & 1, ab);
-                if (!ok) break;
-                tc_fence_after();
-                const int key0 = dq_tile_key0<kSwa>(x, j);
-                const int hi = i - key0;                                   // visible columns: lo <= c <= hi
-                const int lo = kSwa ? max(-key0, hi - W + 1) : 0;
-                const uint32_t ts = tmem + lane_base + bb * 2 * kN;
+        for (int idx = 0; idx < n && ok; ++idx, w.next(p)) {
+            const float2 rec = p.ld[(((long long)w.b * p.Hkv + w.kvh) * p.Tp + w.s * kTok) * 4 + r];
+            const uint64_t nlse2 = f2_pack(-rec.x, -rec.x), nD2 = f2_pack(-rec.y, -rec.y);
+            const int i = w.s * kTok + (r >> 2);
+            const int key0 = w.s * kTok - 128;
+            const int hi = i - key0;                     // visible columns: lo <= c <= hi
+            const int lo = max(-key0, hi - W + 1);
+            ok = warp_wait(bar(C::BS_FULL), idx & 1, ab);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ts = tmem + lane_base + C::kColS, td = tmem + lane_base + C::kColDP;
 #pragma unroll 1
-                for (int c = 0; c < kN / 32; ++c) {
-                    uint32_t s[32], d[32], pk[16];
-                    tmem_ld32(ts + 32 * c, s);
-                    tmem_ld32(ts + kN + 32 * c, d);
-                    tmem_wait_ld();
+            for (int c = 0; c < kSpanBlocks; ++c) {
+                uint32_t sv[32], dv[32], pk[16];
+                tmem_ld32(ts + 32 * c, sv);
+                tmem_ld32(td + 32 * c, dv);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        // two columns per f32x2 instruction (same per-lane rounding)
-                        const int col = 32 * c + e;
-                        const float2 x = f2_unpack(
-                            f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2_2, nlse2));
-                        float p0 = ex2(x.x);
-                        float p1 = ex2(x.y);
-                        p0 = (col >= lo && col <= hi) ? p0 : 0.f;
-                        p1 = (col + 1 >= lo && col + 1 <= hi) ? p1 : 0.f;
-                        const uint64_t dd = f2_add(f2_pack(__uint_as_float(d[e]), __uint_as_float(d[e + 1])), nD2);
-                        const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), dd));
-                        pk[e >> 1] = pack_bf16(ds.x, ds.y);
-                    }
-                    tmem_st16(ts + 16 * c, pk);
+                for (int e = 0; e < 32; e += 2) {
+                    // two columns per f32x2 instruction (same per-lane rounding as the scalar form)
+                    const int col = 32 * c + e;
+                    const float2 x = f2_unpack(
+                        f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2_2, nlse2));
+                    float p0 = ex2(x.x);
+                    float p1 = ex2(x.y);
+                    p0 = (col >= lo && col <= hi) ? p0 : 0.f;
+                    p1 = (col + 1 >= lo && col + 1 <= hi) ? p1 : 0.f;
+                    const uint64_t dd = f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nD2);
+                    const float2 ds = f2_unpack(f2_mul(f2_pack(p0, p1), dd));
+                    pk[e >> 1] = pack_bf16(ds.x, ds.y);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::BDS_READY + bb));
+                // dS of chunk c lands on S columns 16 c .. 16 c + 15 (chunk c / 2, already read)
+                tmem_st16(ts + 16 * c, pk);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::BDS_READY));
         }
     } else if (warp >= 8) {
         // ================================================= epilogue: dq, dw_q
@@ -630,16 +757,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
         float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
+        SwaWalk wk;
+        wk.init(p, u0);
         bool ok = true;
-        QUnit x;
-        for (int k = 0; k < nunits && ok; ++k) {
-            dq_unit_at<kSwa>(p, k, x);
-            ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
+        for (int idx = 0; idx < n && ok; ++idx, wk.next(p)) {
+            ok = warp_wait(bar(C::BACC_FULL), idx & 1, ab);
             if (!ok) break;
             tc_fence_after();
-            const int i = x.qb * 32 + (r >> 2);
+            const int i = wk.s * kTok + (r >> 2);
             const bool valid = i < p.T;
-            const long long off = valid ? (((long long)x.b * p.T + i) * p.Hq + x.kvh * 4 + (r & 3)) * kD : 0;
+            const long long off = valid ? (((long long)wk.b * p.T + i) * p.Hq + wk.kvh * 4 + (r & 3)) * kD : 0;
             norm_rope_backward<R>(tmem + lane_base + C::kColDQ, p.scale, p.x + off, valid, w, p.eps, i, p.theta,
                                   p.dx + off, dwacc);
             tc_fence_before();

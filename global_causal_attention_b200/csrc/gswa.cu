@@ -49,7 +49,7 @@ template <int R>
 bool set_bwd_smem()
 {
     using namespace gswa::bwd;
-    return set_smem(bwd_dq_kernel<R, true>, DqCfg<true>::kSmemBytes) ||
+    return set_smem(bwd_dq_swa_kernel<R>, DqSwaCfg::kSmemBytes) ||
            set_smem(bwd_dq_full_kernel<R>, DqFullCfg::kSmemBytes) ||
            set_smem(bwd_dkdv_kernel<R, true>, KvCfg::kSmemBytes) ||
            set_smem(bwd_dkdv_kernel<R, false>, KvCfg::kSmemBytes);
@@ -291,7 +291,7 @@ void launch_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::
 {
     using namespace gswa::bwd;
     if constexpr (kSwa)
-        bwd_dq_kernel<R, true><<<gq, kThreads, DqCfg<true>::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
+        bwd_dq_swa_kernel<R><<<gq, kThreads, DqSwaCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
     else
         bwd_dq_full_kernel<R><<<gq, kThreads, DqFullCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
     bwd_dkdv_kernel<R, kSwa><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
@@ -373,7 +373,8 @@ int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const
     if (rc != GSWA_OK) return rc;
 
     // 3. dq and dk/dv
-    const int kN = swa ? gswa::bwd::DqCfg<true>::kN : gswa::bwd::DqCfg<false>::kN;
+    // dq kernel's K~/V boxes: 32-key ring blocks (sliding window), 64-key tiles (full causal)
+    const int kN = swa ? gswa::bwd::DqSwaCfg::kTok : gswa::bwd::DqCfg<false>::kN;
     BwdMaps m;
     if (encode_bthd(&m.tq, qt, s->B, s->T, s->Hq, s->D, 4, 32) ||
         encode_bthd(&m.ta, da, s->B, s->T, s->Hq, s->D, 4, 32) ||
