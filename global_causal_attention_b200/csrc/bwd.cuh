@@ -761,12 +761,17 @@ bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         wk.init(p, u0);
         bool ok = true;
         for (int idx = 0; idx < n && ok; ++idx, wk.next(p)) {
-            ok = warp_wait(bar(C::BACC_FULL), idx & 1, ab);
-            if (!ok) break;
-            tc_fence_after();
             const int i = wk.s * kTok + (r >> 2);
             const bool valid = i < p.T;
             const long long off = valid ? (((long long)wk.b * p.T + i) * p.Hq + wk.kvh * 4 + (r & 3)) * kD : 0;
+            // the raw q row (two 128-byte lines) is read twice below: start it toward L2 while dQ~ is computed
+            if (valid) {
+                prefetch_l2(p.x + off);
+                prefetch_l2(p.x + off + 64);
+            }
+            ok = warp_wait(bar(C::BACC_FULL), idx & 1, ab);
+            if (!ok) break;
+            tc_fence_after();
             norm_rope_backward<R>(tmem + lane_base + C::kColDQ, p.scale, p.x + off, valid, w, p.eps, i, p.theta,
                                   p.dx + off, dwacc);
             tc_fence_before();
