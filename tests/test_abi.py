@@ -105,3 +105,35 @@ def test_binding_signatures_match_header(L):
     arity = declared_arity()
     for name, args in L._gswa_signatures.items():
         assert arity[name] == len(args), (name, arity[name], len(args))
+
+
+def _a256(x):
+    return -(-x // 256) * 256
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 64, 4, 1), (2, 100, 8, 2), (8, 4096, 32, 8)])
+def test_workspace_sizes_follow_the_buffer_layouts(B, T, Hq, Hkv):
+    """gswa_workspace_bytes against the layouts the header documents (host
+    code only): bf16 [B,T,H,128] tensors, f32-pair row records [B,Hkv,Tp,4],
+    per-warp dw partials for up to 256 CTAs, each buffer 256-byte aligned."""
+    s = gca.make_shape(B, T, Hq, Hkv)
+    q, k = B * T * Hq * 128 * 2, B * T * Hkv * 128 * 2
+    Tp = -(-T // 32) * 32
+    rec = B * Hkv * Tp * 4 * 8
+    part = _a256(256 * 4 * 128 * 4)
+    assert gca.workspace_bytes(gca.OP_GSWA_FWD, s) == _a256(k)                      # k~
+    assert gca.workspace_bytes(gca.OP_FULL_FWD, s) == _a256(k) + _a256(q)           # k~, q~
+    assert gca.workspace_bytes(gca.OP_GSWA_BWD, s) == _a256(q) + _a256(k) + _a256(q) + _a256(rec) + 2 * part
+    assert gca.workspace_bytes(gca.OP_FULL_BWD, s) == _a256(q) + _a256(k) + _a256(rec) + 2 * part   # no dA
+    assert gca.workspace_bytes(gca.OP_GSWA_DECODE, s) == 0
+
+
+def test_full_decode_workspace_and_the_fixed_scratch():
+    # q~ in f32 [B,Hq,128] + partials [B,Hkv,chunks of 4096 keys,4 heads,(4 + 128) f32]
+    for B, Hq, Hkv, Tmax in [(1, 4, 1, 1), (4, 8, 2, 10000), (32, 32, 8, 262144)]:
+        s = gca.make_shape(B, 1, Hq, Hkv, cache_len=Tmax)
+        nch = -(-Tmax // 4096)
+        want = _a256(B * Hq * 128 * 4) + _a256(B * Hkv * nch * 4 * 132 * 4)
+        assert gca.workspace_bytes(gca.OP_FULL_DECODE, s) == want
+    # the 32-sequence, 262,144-token decode fits the 36 MiB allocation-free scratch
+    assert want <= 36 << 20
