@@ -248,25 +248,17 @@ def build_train(s, dev, seed):
 
 
 def build_prefill(name, s, dev, seed):
-    """The 32-layer attention stack, forward, every layer on the same tensors."""
-    import global_causal_attention_b200 as gca
+    """The 32-layer attention stack, forward, every layer on the same tensors
+    (27 gated-SWA layers and 5 global layers, the schedule of the stack driver)."""
+    from global_causal_attention_b200.stack import AttentionStack
     x = workloads.attention_inputs(s, seed, device=dev)
-    kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
-    sh_full = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, 0, **kw)
-    sh_swa = gca.make_shape(s.B, s.T, s.Hq, s.Hkv, s.D, s.window, **kw)
+    st = AttentionStack(n_layers=LAYERS, window=s.window, rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps,
+                        scale=s.scale)
     y_s, y_f = torch.empty_like(x["q"]), torch.empty_like(x["q"])
     lse = torch.empty(s.B, s.Hq, s.T, dtype=torch.float32, device=dev)
-    ws_ff = _ws(gca, gca.OP_FULL_FWD, sh_full, dev)
-    ws_sf = _ws(gca, gca.OP_GSWA_FWD, sh_swa, dev)
-    q, k, v, g, wq, wk = (x[n] for n in ("q", "k", "v", "g", "wq", "wk"))
-    calls = []
-    for layer in range(1, LAYERS + 1):
-        if workloads.layer_is_global(layer):
-            calls.append(("full_attn_fwd", lambda: gca.full_attn_fwd(q, k, v, wq, wk, y=y_f, lse=lse,
-                                                                     workspace=ws_ff, **kw)))
-        else:
-            calls.append(("gswa_fwd", lambda: gca.gswa_fwd(q, k, v, g, wq, wk, window=s.window, y=y_s, lse=lse,
-                                                           workspace=ws_sf, **kw)))
+    outs = [(y_f, lse) if st.is_global(l) else (y_s, lse) for l in range(1, LAYERS + 1)]
+    ws = st.prefill_workspace(s.B, s.T, s.Hq, s.Hkv, dev)
+    calls = st.prefill_calls(x, outs, workspace=ws)
     return Step(name, s, s.B * s.T, calls, x, [y_s])
 
 
@@ -275,34 +267,35 @@ def build_decode(dev, seed):
     global layers read one 262,144-token linear cache (34 GB of K/V; five
     distinct caches would not fit in HBM, and a cache this size streams from
     HBM either way); every SWA layer has its own 128-slot ring."""
-    import global_causal_attention_b200 as gca
+    from global_causal_attention_b200.stack import AttentionStack
     d = workloads.DECODE_256K
     B, Hq, Hkv, D, W, Tmax = d["B"], d["Hq"], d["Hkv"], d["D"], d["window"], d["Tmax"]
     s = workloads.Shape(B=B, T=1, Hq=Hq, Hkv=Hkv, window=W, rope_base=d["rope_base"])
-    kw = dict(rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps, scale=s.scale)
+    st = AttentionStack(n_layers=LAYERS, window=W, rope_dims=s.rope_dims, rope_base=s.rope_base, eps=s.eps,
+                        scale=s.scale)
     bf = dict(dtype=torch.bfloat16, device=dev)
     kc = workloads.fill_randn_bf16_(torch.empty(B, Hkv, Tmax, D, **bf), seed * 100 + 1)
     vc = workloads.fill_randn_bf16_(torch.empty(B, Hkv, Tmax, D, **bf), seed * 100 + 2)
     pos = torch.full((B,), d["pos"], dtype=torch.int64, device=dev)
     wq = torch.ones(D, **bf)
     wk = torch.ones(D, **bf)
-    ws_fd = _ws(gca, gca.OP_FULL_DECODE, gca.make_shape(B, 1, Hq, Hkv, D, W, cache_len=Tmax, **kw), dev)
-    calls, h2d, y = [], {"pos": pos}, None
+    ins, caches, outs, h2d = [], [], [], {"pos": pos}
     for layer in range(1, LAYERS + 1):
         li = workloads.decode_inputs(B, Hq, Hkv, D, 1, seed=seed * 64 + layer, device=dev)
-        q, k, v, g = li["q"], li["k"], li["v"], li["g"]
+        x = {n: li[n] for n in ("q", "k", "v", "g")}
+        x.update(wq=wq, wk=wk)
         for n in ("q", "k", "v", "g"):
             h2d[f"{n}{layer}"] = li[n]
-        y = torch.empty_like(q)
-        if workloads.layer_is_global(layer):
-            calls.append(("full_decode", lambda q=q, k=k, v=v, y=y: gca.full_decode(
-                q, k, v, wq, wk, kc, vc, pos, y=y, workspace=ws_fd, **kw)))
+        ins.append(x)
+        outs.append(torch.empty_like(li["q"]))
+        if st.is_global(layer):
+            caches.append((kc, vc))
         else:
-            kr = workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 10 + layer)
-            vr = workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 50 + layer)
-            calls.append(("gswa_decode", lambda q=q, k=k, v=v, g=g, kr=kr, vr=vr, y=y: gca.gswa_decode(
-                q, k, v, g, wq, wk, kr, vr, pos, y=y, **kw)))
-    return Step("decode_256k", s, B, calls, h2d, [y], pos=d["pos"])
+            caches.append((workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 10 + layer),
+                           workloads.fill_randn_bf16_(torch.empty(B, Hkv, W, D, **bf), seed * 100 + 50 + layer)))
+    ws = st.decode_workspace(B, Hq, Hkv, Tmax, dev)
+    calls = st.decode_calls(ins, caches, pos, outs, workspace=ws)
+    return Step("decode_256k", s, B, calls, h2d, [outs[-1]], pos=d["pos"])
 
 
 def build(name, dev, seed):
@@ -418,20 +411,38 @@ def time_e2e(steps, host_in, host_out, K, W, stream, dist_on):
     return ms
 
 
-def op_table(step, op_ms, K, pk):
-    """Per entry point: calls per step, ms per call, achieved rate against its bound."""
+def tensor_peak(pk, clocks, timed_s):
+    """(peak TFLOP/s, which) for the tensor-bound entry points of this run: the
+    burst peak (cuBLAS measured in isolation at full clocks) when the timed
+    region is short (< 1 s) or ran at full clocks without the power cap, the
+    sustained peak (cuBLAS in a seconds-long loop under the power cap)
+    otherwise."""
+    full_clock = clocks is not None and clocks["sm_mhz"] >= 0.98 * clocks["sm_max_mhz"]
+    capped = clocks is not None and "sw_power_cap" in clocks["reasons"]
+    if timed_s < 1.0 or (full_clock and not capped):
+        return pk["bf16_tflops"], "burst"
+    return pk["bf16_tflops_sustained"], "sustained"
+
+
+def op_table(step, op_ms, K, pk, tpeak):
+    """Per entry point: calls per step, ms per call, achieved rate against its
+    bound.  Tensor-bound calls carry the fraction of both tensor peaks."""
     table = {}
     for op in step.ops():
         n = sum(1 for o, _ in step.calls if o == op)
         per_call = op_ms[op] / (K * n)
         bound, amount, unit = algorithmic_work(op, step.s, step.pos)
+        e = {"calls_per_step": n, "ms_per_call": per_call, "bound": bound, "unit": unit,
+             "algorithmic_per_call": amount, "launches_per_call": LAUNCHES[op]}
         if bound == "hbm":
-            achieved, peak = amount / (per_call / 1e3) / 1e9, pk["hbm_gbs"]
+            achieved = amount / (per_call / 1e3) / 1e9
+            e.update(achieved=achieved, peak=pk["hbm_gbs"], frac=achieved / pk["hbm_gbs"])
         else:
-            achieved, peak = amount / (per_call / 1e3) / 1e12, pk["bf16_tflops_sustained"]
-        table[op] = {"calls_per_step": n, "ms_per_call": per_call, "bound": bound, "achieved": achieved,
-                     "unit": unit, "peak": peak, "frac": achieved / peak,
-                     "algorithmic_per_call": amount, "launches_per_call": LAUNCHES[op]}
+            achieved = amount / (per_call / 1e3) / 1e12
+            e.update(achieved=achieved, peak=tpeak[0], peak_kind=tpeak[1], frac=achieved / tpeak[0],
+                     frac_burst=achieved / pk["bf16_tflops"],
+                     frac_sustained=achieved / pk["bf16_tflops_sustained"])
+        table[op] = e
     return table
 
 
@@ -459,10 +470,14 @@ def oracle_sample(name, budget_s):
     cores = _oracle_cores()
     if name == "train_4k":
         s = WORKLOADS["train_4k"]
-        # one sequence's causal prefix of T' tokens over G' KV groups: the outputs of a
-        # prefix depend on the prefix only, so this is an exact slice of the step
-        G = max(1, min(s.Hkv, cores)) if budget_s >= 10 else 1
-        Tp = s.T if budget_s >= 10 else max(128, min(s.T, int(math.sqrt(budget_s / 1.1e-6)) // 128 * 128))
+        # one sequence's causal prefix of T' tokens over G KV groups: the outputs of a
+        # prefix depend on the prefix only, so this is an exact slice of the step.
+        # G covers every host core the oracle can use (it runs the KV groups on
+        # separate threads); the prefix shrinks to fit the budget: with one
+        # group per thread the whole 4,096-token prefix takes about 20 s, the
+        # full causal part (most of it) growing as T'^2.
+        G = max(1, min(s.Hkv, cores))
+        Tp = s.T if budget_s >= 20.0 else max(128, int(s.T * math.sqrt(budget_s / 20.0)) // 128 * 128)
         sg = s.replace(B=1, T=Tp, Hq=4 * G, Hkv=G)
         x = _memo(("train", Tp, G), lambda: workloads.attention_inputs(sg, 0, with_grad=True))
         kw = oracle.shape_kwargs(sg)
@@ -594,6 +609,37 @@ def workload_config(name, n):
 
 
 DEFAULT_STEPS = {"train_4k": 100, "prefill_64k": 5, "prefill_256k": 2, "decode_256k": 30}
+# Steps of the other workloads that a default (train_4k) run also times.
+EXTRA_STEPS = {"prefill_64k": 4, "prefill_256k": 2, "decode_256k": 20}
+EXTRA_WARMUP = {"prefill_64k": 3, "prefill_256k": 3, "decode_256k": 3}
+
+
+def measure(name, dev, seed, steps, warmup, stream, dist_on, pk):
+    """Build workload `name`, time `steps` steps after `warmup` (clocks sampled),
+    and return (step, ms, clocks, per-entry-point table, roofline of the
+    dominant entry point)."""
+    import global_causal_attention_b200 as gca
+    step = build(name, dev, seed=seed)
+    clk = ClockSampler(torch.cuda.current_device())
+    ms, op_ms = time_steps(step, steps, warmup, stream, dist_on, sampler=clk, per_op=True)
+    clocks = clk.summary()
+    if gca.gswa_check_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait or a bad position")
+    tpeak = tensor_peak(pk, clocks, ms / 1e3)
+    ops = op_table(step, op_ms, steps, pk, tpeak)
+    for o in ops:
+        ops[o]["traffic"] = TRAFFIC.get((name, o))
+    dom = max(ops, key=lambda o: ops[o]["ms_per_call"] * ops[o]["calls_per_step"])
+    d = ops[dom]
+    roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
+                "frac": d["frac"], "traffic": d["traffic"], "kernel": dom,
+                "launches": d["launches_per_call"], "ms_per_launch": d["ms_per_call"],
+                "algorithmic_per_launch": d["algorithmic_per_call"],
+                "peak_source": pk["source"] + (f" {d['peak_kind']}" if d["bound"] == "tensor" else "")}
+    if d["bound"] == "tensor":
+        roofline["frac_burst"] = d["frac_burst"]
+        roofline["frac_sustained"] = d["frac_sustained"]
+    return step, ms, clocks, ops, roofline
 
 
 def main():
@@ -604,6 +650,8 @@ def main():
     ap.add_argument("--workload", default="train_4k", choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads' device timings that the default train_4k run adds")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]
@@ -624,28 +672,12 @@ def main():
 
     import global_causal_attention_b200 as gca
     gca.lib()
-    step = build(args.workload, dev, seed=rank)
+    pk = peaks()
     stream = torch.cuda.current_stream(dev)
-
-    clk = ClockSampler(torch.cuda.current_device())
-    ms, op_ms = time_steps(step, args.steps, args.warmup, stream, dist_on, sampler=clk, per_op=True)
-    clocks = clk.summary()
-    if gca.gswa_check_status() != 0:
-        raise RuntimeError("device status reports a timed-out wait or a bad position")
+    step, ms, clocks, ops, roofline = measure(args.workload, dev, rank, args.steps, args.warmup, stream, dist_on,
+                                              pk)
     tokens = step.tokens * world
     value = tokens * args.steps / (ms / 1e3)
-
-    pk = peaks()
-    ops = op_table(step, op_ms, args.steps, pk)
-    for o in ops:
-        ops[o]["traffic"] = TRAFFIC.get((args.workload, o))
-    dom = max(ops, key=lambda o: ops[o]["ms_per_call"] * ops[o]["calls_per_step"])
-    d = ops[dom]
-    roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-                "frac": d["frac"], "traffic": TRAFFIC.get((args.workload, dom)), "kernel": dom,
-                "launches": d["launches_per_call"], "ms_per_launch": d["ms_per_call"],
-                "algorithmic_per_launch": d["algorithmic_per_call"],
-                "peak_source": pk["source"] + (" sustained" if d["bound"] == "tensor" else "")}
 
     # End to end through the public API: every step's inputs copied from pinned
     # host memory to the device and its outputs back to pinned host memory,
@@ -664,6 +696,28 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, step.tokens)
 
+    # The other workloads, timed the same way in the same run (one GPU only):
+    # their device time, per-entry-point table and roofline.
+    launches = step.launches() * args.steps
+    extra = None
+    if world == 1 and args.workload == "train_4k" and not args.no_extra:
+        del step, host_in, host_out
+        extra = {}
+        for name in WORKLOAD_NAMES:
+            if name == args.workload:
+                continue
+            torch.cuda.empty_cache()
+            st2, ms2, clk2, ops2, roof2 = measure(name, dev, rank, EXTRA_STEPS[name], EXTRA_WARMUP[name], stream,
+                                                  False, pk)
+            extra[name] = {"steps": EXTRA_STEPS[name], "warmup": EXTRA_WARMUP[name],
+                           "ms_per_step": ms2 / EXTRA_STEPS[name],
+                           "value": st2.tokens * EXTRA_STEPS[name] / (ms2 / 1e3), "unit": UNIT,
+                           "config": workload_config(name, 1)["workload"], "roofline": roof2, "ops": ops2,
+                           "gpu_launches": st2.launches() * EXTRA_STEPS[name], "clocks": clk2}
+            del st2
+        if gca.gswa_check_status() != 0:
+            raise RuntimeError("device status reports a timed-out wait or a bad position")
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -673,10 +727,12 @@ def main():
             "roofline": roofline,
             "ops": ops,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": step.launches() * args.steps,
+            "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
+        if extra is not None:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
     if dist_on:
         torch.distributed.barrier()

@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
   gswa_bwd, full_attn_bwd, gswa_decode, full_decode  (see include/gswa.h)
   gswa_kv_cache_bytes  KV-cache footprint closed form (§2.3)
   gswa_check_status    read and clear the device status word
+  gswa_set_wait_limit_ns  lower the kernels' bounded-wait limit (failure tests)
 """
 from __future__ import annotations
 
@@ -77,6 +78,8 @@ def lib():
         L.gswa_kv_cache_bytes.restype = ctypes.c_int64
         L.gswa_check_status.argtypes = [P]
         L.gswa_check_status.restype = I
+        L.gswa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.gswa_set_wait_limit_ns.restype = I
         L.gswa_strerror.argtypes = [I]
         L.gswa_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -282,3 +285,9 @@ def gswa_kv_cache_bytes(n_global_layers, n_window_layers, window, Hkv, D, bytes_
 def gswa_check_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(lib().gswa_check_status(_stream(stream)))
+
+
+def gswa_set_wait_limit_ns(ns: int) -> None:
+    """Make every bounded wait inside the kernels give up after `ns` ns on the
+    current device (0 restores the default 4 s); for failure-detection tests."""
+    _check(lib().gswa_set_wait_limit_ns(int(ns)), "gswa_set_wait_limit_ns")

@@ -167,7 +167,11 @@ swa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(tile + off), "r"(bits.x), "r"(bits.y) : "memory");
     }
     __syncthreads();
-    if (!landed) return;
+    if (!landed) {
+        // the wait gave up: the ring's copy must still land before the CTA exits
+        if (threadIdx.x == 0) swa::drain_wait(bar, 0);
+        return;
+    }
 
     // scores: lane owns slots lane + 32 i; slot s holds position pos - ((slot_new - s) mod W)
     float sc[4];

@@ -230,8 +230,7 @@ int launch_qk_prep(const gswa_shape_t *s, int H, const void *x, const void *w, v
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GSWA_NOALLOC_SCRATCH_BYTES];
 
 struct NoAllocDevice {
-    bool ready = false;
-    int status = GSWA_OK;
+    bool ready = false;       // set once the lookup succeeded
     void *scratch = nullptr;
 };
 NoAllocDevice g_noalloc[kMaxDevices];
@@ -245,16 +244,20 @@ int noalloc_scratch(void **scratch)
     std::lock_guard<std::mutex> lock(g_mutex);
     NoAllocDevice &d = g_noalloc[dev];
     if (!d.ready) {
-        d.ready = true;
         void *ptr = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess || ptr == nullptr)
-            d.status = GSWA_ERR_LAUNCH;
-        else
-            d.scratch = ptr;
+        if (e != cudaSuccess || ptr == nullptr) {
+            // not cached: clear the runtime's error state so that a later call
+            // (say, one made outside a stream capture) can try again
+            (void)cudaGetLastError();
+            *scratch = nullptr;
+            return GSWA_ERR_LAUNCH;
+        }
+        d.scratch = ptr;
+        d.ready = true;
     }
     *scratch = d.scratch;
-    return d.status;
+    return GSWA_OK;
 }
 
 // Backward workspace: prepared q~ [B,T,Hq,D] and k~ [B,T,Hkv,D] (bf16),
@@ -431,6 +434,57 @@ int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const
     const unsigned rt = gswa::bwd::kD * gswa::bwd::kReduceSlices;
     gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_q, (int)gq * 4, dw_q);
     gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_k, (int)gk * 4, dw_k);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
+// Argument checks of full_decode and full_decode_noalloc (everything but the
+// scratch they run on).
+int check_full_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *w_q,
+                      const void *w_k, const void *k_cache, const void *v_cache, const int64_t *pos,
+                      const void *y)
+{
+    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->cache_len < 1) return GSWA_ERR_INVALID_ARG;
+    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
+    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
+        return GSWA_ERR_UNSUPPORTED_SHAPE;
+    if (s->B == 0) return GSWA_OK;
+    if (!q || !k || !v || !w_q || !w_k || !k_cache || !v_cache || !pos || !y) return GSWA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
+        return GSWA_ERR_MISALIGNED;
+    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
+    if (cache_rows + gswa::dec::kStageKeys > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;   // TMA row coordinates
+    return GSWA_OK;
+}
+
+// The three launches of a full-cache decode step, on `scratch` laid out as
+// full_decode_ws() describes: q~ [B, Hq, D] f32, then the chunk partials.
+int launch_full_decode(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *w_q,
+                       const void *w_k, void *k_cache, void *v_cache, const int64_t *pos, void *y, void *scratch,
+                       cudaStream_t st)
+{
+    gswa::dec::Params p;
+    fill_dec(p, s);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    p.pos = pos;
+    p.y = static_cast<__nv_bfloat16 *>(y);
+    p.qt = static_cast<float *>(scratch);
+    p.part = reinterpret_cast<float *>(static_cast<char *>(scratch) + align256((size_t)s->B * s->Hq * s->D * 4));
+    CUtensorMap tkc, tvc;
+    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
+    if (encode_rows(&tkc, k_cache, cache_rows, gswa::dec::kStageKeys) ||
+        encode_rows(&tvc, v_cache, cache_rows, gswa::dec::kStageKeys))
+        return GSWA_ERR_INVALID_ARG;
+    gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
+    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkThreads,
+                                          gswa::dec::kDecSmemBytes, st>>>(tkc, tvc, p);
+    gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
@@ -633,97 +687,33 @@ int full_decode(const gswa_shape_t *s, const void *q, const void *k, const void 
                 const int64_t *pos, void *y, void *workspace, size_t workspace_bytes,
                 void *stream)
 {
-    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->cache_len < 1) return GSWA_ERR_INVALID_ARG;
-    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
-    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
-        return GSWA_ERR_UNSUPPORTED_SHAPE;
-    if (s->B == 0) return GSWA_OK;
-    if (!q || !k || !v || !w_q || !w_k || !k_cache || !v_cache || !pos || !y) return GSWA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
-        return GSWA_ERR_MISALIGNED;
+    int rc = check_full_decode(s, q, k, v, w_q, w_k, k_cache, v_cache, pos, y);
+    if (rc != GSWA_OK || s->B == 0) return rc;
     if (workspace == nullptr || workspace_bytes < full_decode_ws(s)) return GSWA_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
     int num_sms = 0;
-    int rc = device_setup(&num_sms);
+    rc = device_setup(&num_sms);
     if (rc != GSWA_OK) return rc;
-    gswa::dec::Params p;
-    fill_dec(p, s);
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
-    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
-    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
-    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
-    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
-    p.pos = pos;
-    p.y = static_cast<__nv_bfloat16 *>(y);
-    p.qt = static_cast<float *>(workspace);
-    p.part = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                       align256((size_t)s->B * s->Hq * s->D * 4));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // cache rows as TMA coordinates (32-bit)
-    CUtensorMap tkc, tvc;
-    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
-    if (cache_rows + gswa::dec::kStageKeys > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;
-    if (encode_rows(&tkc, k_cache, cache_rows, gswa::dec::kStageKeys) ||
-        encode_rows(&tvc, v_cache, cache_rows, gswa::dec::kStageKeys))
-        return GSWA_ERR_INVALID_ARG;
-    gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
-    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkThreads,
-                                          gswa::dec::kDecSmemBytes, st>>>(tkc, tvc, p);
-    gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+    return launch_full_decode(s, q, k, v, w_q, w_k, k_cache, v_cache, pos, y, workspace,
+                              static_cast<cudaStream_t>(stream));
 }
 
 int full_decode_noalloc(const gswa_shape_t *s, const void *q, const void *k, const void *v,
                         const void *w_q, const void *w_k, void *k_cache, void *v_cache,
                         const int64_t *pos, void *y, void *stream)
 {
-    if (s == nullptr || s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->cache_len < 1) return GSWA_ERR_INVALID_ARG;
-    if (!(s->eps >= 0.f) || !(s->rope_base > 0.0) || !std::isfinite(s->scale)) return GSWA_ERR_INVALID_ARG;
-    if (s->D != 128 || s->Hq != 4 * s->Hkv || s->rope_dims < 0 || s->rope_dims > s->D || (s->rope_dims & 1))
-        return GSWA_ERR_UNSUPPORTED_SHAPE;
-    if (s->B == 0) return GSWA_OK;
-    if (!q || !k || !v || !w_q || !w_k || !k_cache || !v_cache || !pos || !y) return GSWA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 7u))
-        return GSWA_ERR_MISALIGNED;
+    int rc = check_full_decode(s, q, k, v, w_q, w_k, k_cache, v_cache, pos, y);
+    if (rc != GSWA_OK || s->B == 0) return rc;
     // the same scratch layout full_decode takes from its workspace
-    const size_t q_bytes = align256((size_t)s->B * s->Hq * s->D * 4);
     if (full_decode_ws(s) > GSWA_NOALLOC_SCRATCH_BYTES) return GSWA_ERR_SCRATCH_LIMIT;
     int num_sms = 0;
-    int rc = device_setup(&num_sms);
+    rc = device_setup(&num_sms);
     if (rc != GSWA_OK) return rc;
     void *scratch = nullptr;
     rc = noalloc_scratch(&scratch);
     if (rc != GSWA_OK) return rc;
-    gswa::dec::Params p;
-    fill_dec(p, s);
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
-    p.wq = static_cast<const __nv_bfloat16 *>(w_q);
-    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
-    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
-    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
-    p.pos = pos;
-    p.y = static_cast<__nv_bfloat16 *>(y);
-    p.qt = static_cast<float *>(scratch);
-    p.part = reinterpret_cast<float *>(static_cast<char *>(scratch) + q_bytes);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // cache rows as TMA coordinates (32-bit)
-    CUtensorMap tkc, tvc;
-    const long long cache_rows = (long long)s->B * s->Hkv * s->cache_len;
-    if (cache_rows + gswa::dec::kStageKeys > 0x7fffffffLL) return GSWA_ERR_UNSUPPORTED_SHAPE;
-    if (encode_rows(&tkc, k_cache, cache_rows, gswa::dec::kStageKeys) ||
-        encode_rows(&tvc, v_cache, cache_rows, gswa::dec::kStageKeys))
-        return GSWA_ERR_INVALID_ARG;
-    gswa::dec::full_decode_prep_kernel<<<s->B * s->Hkv, 128, 0, st>>>(p);
-    gswa::dec::full_decode_chunk_kernel<<<dim3(p.nchunks, s->B * s->Hkv), gswa::dec::kChunkThreads,
-                                          gswa::dec::kDecSmemBytes, st>>>(tkc, tvc, p);
-    gswa::dec::full_decode_combine_kernel<<<s->B * s->Hq, gswa::dec::kD, 0, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+    return launch_full_decode(s, q, k, v, w_q, w_k, k_cache, v_cache, pos, y, scratch,
+                              static_cast<cudaStream_t>(stream));
 }
 
 size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
@@ -761,6 +751,13 @@ int gswa_check_status(void *stream)
         return v == gswa::kStatusBadArg ? GSWA_ERR_INVALID_ARG : GSWA_ERR_TIMEOUT;
     }
     return GSWA_OK;
+}
+
+int gswa_set_wait_limit_ns(uint64_t ns)
+{
+    const unsigned long long v = ns == 0 ? gswa::kWaitLimitNs : (unsigned long long)ns;
+    if (cudaMemcpyToSymbol(gswa::g_wait_limit_ns, &v, sizeof v) != cudaSuccess) return GSWA_ERR_LAUNCH;
+    return cudaDeviceSynchronize() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
 }
 
 const char *gswa_strerror(int code)

@@ -19,6 +19,10 @@ constexpr int kStatusBadArg = 2;   // a device-side argument (a decode position)
 // A wait gives up after this much wall time (the kernels' longest legitimate
 // wait is a few microseconds; profilers that serialise passes stay far below).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// The limit the kernels apply: kWaitLimitNs unless gswa_set_wait_limit_ns()
+// lowered it (a failure-detection test makes waits give up this way).  Read
+// only once a wait has already spun, so it costs nothing on the fast path.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -119,7 +123,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
         if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
         if ((spin & 3u) == 3u) {
             if (ab.raised()) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > g_wait_limit_ns) {
                 ab.raise(kStatusTimeout);
                 return false;
             }
@@ -131,7 +135,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
 // turn): call tick(progressed) once per pass.  The wall clock is a slow read,
 // so it is consulted only every 512 idle passes.  Returns false (with the
 // CTA's abort flag raised) once the loop has made no progress for
-// kWaitLimitNs, or when another role raised the flag.
+// g_wait_limit_ns, or when another role raised the flag.
 struct PollWatch {
     uint32_t idle = 0;
     uint64_t t0 = 0;
@@ -148,7 +152,7 @@ struct PollWatch {
             t0 = now;
             return true;
         }
-        if (now - t0 > kWaitLimitNs) {
+        if (now - t0 > g_wait_limit_ns) {
             ab.raise(kStatusTimeout);
             return false;
         }

@@ -106,16 +106,34 @@ int full_attn_fwd(const gswa_shape_t *shape, const void *q, const void *k, const
                   size_t workspace_bytes, void *stream);
 
 /*
- * Backward of gswa_fwd.  Reads q, k, v, g, w_q, w_k, the forward's y and lse,
- * and the upstream gradient dy [B,T,Hq,D]; writes dq, dg [B,T,Hq,D],
- * dk, dv [B,T,Hkv,D] (bf16) and dw_q, dw_k [D] (f32).  All device.
+ * Backward of gswa_fwd: the gradients a training step of the gated-SWA layers
+ * needs (ZGCM-1 §2.2 hybrid-attention experiments, whose models are trained
+ * at sequence length 4,096; §3.1 pre-training hyperparameters).  With
+ * σ = sigmoid(g), A = y / σ and the forward's P:
+ *   dA = dy ⊙ σ, dg = dy ⊙ y ⊙ (1 - σ), D_i = Σ_d dy_i y_i,
+ *   dV = Σ_heads P^T dA, dS = P ⊙ (dA V^T - D), dq~ = scale dS K~,
+ *   dk~ = scale Σ_heads dS^T Q~, then back through RoPE (the transposed
+ *   rotation) and RMSNorm to dq, dk, dw_q, dw_k.
+ *   Reads q, k, v, g, w_q, w_k, the forward's y and lse (as gswa_fwd wrote
+ *   them; the softmax is recomputed from lse, not stored), and the upstream
+ *   gradient dy [B,T,Hq,D].  Writes dq, dg [B,T,Hq,D], dk, dv [B,T,Hkv,D]
+ *   (bf16) and dw_q, dw_k [D] (f32, summed over every token and head).  All
+ *   device.  workspace: gswa_workspace_bytes(GSWA_OP_GSWA_BWD) bytes (device,
+ *   16-byte aligned), overwritten.  Results are bitwise reproducible.
+ *   B * T = 0 writes zero weight gradients and nothing else.
  */
 int gswa_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
              const void *g, const void *w_q, const void *w_k, const void *y, const float *lse,
              const void *dy, void *dq, void *dk, void *dv, void *dg, float *dw_q, float *dw_k,
              void *workspace, size_t workspace_bytes, void *stream);
 
-/* Backward of full_attn_fwd (no gate, no dg). */
+/*
+ * Backward of full_attn_fwd, the global layers' share of a training step
+ * (ZGCM-1 §2.1: global layers attend over the whole causal context, no gate;
+ * §2.2 and §3.1 as for gswa_bwd).  The formulas of gswa_bwd with σ = 1
+ * (dA = dy) over every key j <= i; no g, no dg.  Layouts, workspace
+ * (gswa_workspace_bytes(GSWA_OP_FULL_BWD)) and ownership as for gswa_bwd.
+ */
 int full_attn_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                   const void *w_q, const void *w_k, const void *y, const float *lse,
                   const void *dy, void *dq, void *dk, void *dv, float *dw_q, float *dw_k,
@@ -217,6 +235,18 @@ int64_t gswa_kv_cache_bytes(int n_global_layers, int n_window_layers, int window
  * GSWA_ERR_LAUNCH on a CUDA error.
  */
 int gswa_check_status(void *stream);
+
+/*
+ * Failure-detection hook: every bounded wait inside the kernels of this
+ * library gives up after `ns` nanoseconds of wall time on the current device
+ * instead of the default 4 s (ns = 0 restores the default).  A kernel whose
+ * wait gives up stops all of its roles, lets its in-flight copies land,
+ * frees its tensor memory and returns; gswa_check_status() then reports
+ * GSWA_ERR_TIMEOUT and the outputs of that call are undefined.  Meant for
+ * tests that exercise that path; synchronous (it waits for the device).
+ * Returns GSWA_OK or GSWA_ERR_LAUNCH.
+ */
+int gswa_set_wait_limit_ns(uint64_t ns);
 
 /* Human-readable name of a return code (static string). */
 const char *gswa_strerror(int code);

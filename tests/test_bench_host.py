@@ -65,13 +65,16 @@ def test_op_table_fraction():
     step = bench.Step("t", s, s.B * s.T, [("gswa_fwd", None), ("full_attn_fwd", None), ("gswa_fwd", None)], {}, [])
     K = 4
     op_ms = {"gswa_fwd": 2 * K * 0.5, "full_attn_fwd": K * 2.0}   # 0.5 ms and 2.0 ms per call
-    pk = dict(hbm_gbs=6536.7, bf16_tflops_sustained=1387.5)
-    t = bench.op_table(step, op_ms, K, pk)
+    pk = dict(hbm_gbs=6536.7, bf16_tflops=1656.9, bf16_tflops_sustained=1387.5)
+    t = bench.op_table(step, op_ms, K, pk, (1656.9, "burst"))
     assert t["gswa_fwd"]["calls_per_step"] == 2
     assert t["gswa_fwd"]["achieved"] == pytest.approx(943_718_400 / 0.5e-3 / 1e9)
     assert t["gswa_fwd"]["frac"] == pytest.approx(943_718_400 / 0.5e-3 / 1e9 / 6536.7)
-    assert t["full_attn_fwd"]["achieved"] == pytest.approx(1_099_780_063_232 / 2.0e-3 / 1e12)
-    assert t["full_attn_fwd"]["frac"] == pytest.approx(1_099_780_063_232 / 2.0e-3 / 1e12 / 1387.5)
+    tf = 1_099_780_063_232 / 2.0e-3 / 1e12
+    assert t["full_attn_fwd"]["achieved"] == pytest.approx(tf)
+    assert t["full_attn_fwd"]["frac"] == pytest.approx(tf / 1656.9)
+    assert t["full_attn_fwd"]["frac_burst"] == pytest.approx(tf / 1656.9)
+    assert t["full_attn_fwd"]["frac_sustained"] == pytest.approx(tf / 1387.5)
     assert step.launches() == 2 * bench.LAUNCHES["gswa_fwd"] + bench.LAUNCHES["full_attn_fwd"]
 
 
@@ -79,3 +82,31 @@ def test_every_entry_point_has_a_launch_count():
     ops = {"gswa_fwd", "gswa_bwd", "full_attn_fwd", "full_attn_bwd", "gswa_decode", "full_decode"}
     assert set(bench.LAUNCHES) == ops
     assert all(n >= 1 for n in bench.LAUNCHES.values())
+
+
+def test_tensor_peak_follows_the_clocks():
+    """Burst peak for a short region or a run at full clocks without the power
+    cap; the sustained (power-capped) peak for a long run that hit the cap."""
+    pk = dict(bf16_tflops=1656.9, bf16_tflops_sustained=1387.5)
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(pk, full, 5.0) == (1656.9, "burst")
+    assert bench.tensor_peak(pk, capped, 0.2) == (1656.9, "burst")
+    assert bench.tensor_peak(pk, capped, 5.0) == (1387.5, "sustained")
+    assert bench.tensor_peak(pk, None, 5.0) == (1387.5, "sustained")
+
+
+def test_stack_schedules():
+    """ZGCM-1 §2.1: 32 layers, global at 1-based 6, 12, 18, 24, 30 (Figure 3
+    caption: the last global layer is 29 counted from 0); §2.2's 1:1 and 3:1
+    schedules put a global layer after every one or three SWA layers."""
+    from global_causal_attention_b200.stack import AttentionStack, global_layers
+    assert global_layers(32, 5) == workloads.GLOBAL_LAYERS_1BASED == (6, 12, 18, 24, 30)
+    assert max(global_layers(32, 5)) - 1 == 29
+    assert global_layers(32, 3) == tuple(range(4, 33, 4))
+    assert global_layers(32, 1) == tuple(range(2, 33, 2))
+    st = AttentionStack()
+    kinds = st.kinds()
+    assert kinds.count("global") == 5 and kinds.count("swa") == 27
+    assert kinds[30:] == ["swa", "swa"]
+    assert all(st.is_global(l) == workloads.layer_is_global(l) for l in range(1, 33))

@@ -84,3 +84,27 @@ def test_swa_fwd_full_size_sampled_rows(workload, nrows):
                              gated=True, rows=rows.numpy(), **oracle.shape_kwargs(s))
     assert_fwd_close(y[:, rows.cuda()], yo, "y")
     assert_fwd_close(lse[:, :, rows.cuda()], lo, "lse")
+
+
+def test_gate_precision_window_1():
+    """With window 1 each row attends to its own key only (P = 1), so the
+    kernel's output is bf16(v ⊙ σ~(g)) and its error against the exact
+    v ⊙ σ(g) is the gate's evaluation error plus the final bf16 rounding.
+    The kernel evaluates σ on f16 pairs (one tanh.approx.f16x2 per pair);
+    this measures what that costs next to the unavoidable rounding of the
+    output to bf16, and bounds it."""
+    s = Shape(B=2, T=2048, Hq=8, Hkv=2, window=1)
+    x = attention_inputs(s, 21)
+    y, _ = run_gpu(s, x)
+    v = x["v"].double().repeat_interleave(4, dim=2)
+    exact = v * torch.sigmoid(x["g"].double())
+    best = exact.to(torch.bfloat16).double()          # the exact value, rounded once to bf16
+    yd = y.double().cpu()
+    nrm = exact.norm().item()
+    e_gpu = (yd - exact).norm().item() / nrm
+    e_round = (best - exact).norm().item() / nrm
+    e_gate = (yd - best).norm().item() / nrm
+    print(f"gate precision: rel-L2 vs exact {e_gpu:.3e}; bf16 rounding alone {e_round:.3e}; "
+          f"gate evaluation {e_gate:.3e}; max |y - exact| {(yd - exact).abs().max().item():.3e}")
+    assert e_gpu <= 5e-3
+    assert e_gate <= 2e-3
