@@ -1,5 +1,5 @@
-// bwd.cuh -- backward of the attention core (gated sliding window and full
-// causal), for sm_100a.
+// bwd.cuh -- backward of the gated sliding-window attention core, and the
+// pieces the full causal backward (bwd_full.cuh) shares with it, for sm_100a.
 //
 // The forward (ZGCM-1 §2.1, Figure 3 caption) is, per query row i of head h
 // (kv head h / 4), with q~ = RoPE(RMSNorm(q) w_q), k~ = RoPE(RMSNorm(k) w_k):
@@ -14,17 +14,16 @@
 //
 // Kernels:
 //   bwd_prep     per row: D and lse log2 e into a row-ordered record, dA and
-//                dg (gated only)
-//   bwd_dq_swa / bwd_dq_full
-//                query-stationary (M = 128 rows = 4 heads x 32 tokens): S =
-//                Q~K~^T and dP = dA V^T into TMEM (sliding window: the unit's
-//                160-key span from K~/V rings kept across consecutive units;
-//                full: 64-key tiles); P from the forward's lse; dS (bf16);
-//                dQ~ += dS K~ in TMEM; epilogue: RoPE^T and the RMSNorm
-//                backward against the raw q, per-warp dw_q partials
+//                dg (gated only); shared with the full causal backward
+//   bwd_dq_swa   query-stationary (M = 128 rows = 4 heads x 32 tokens): S =
+//                Q~K~^T and dP = dA V^T into TMEM over the unit's 160-key
+//                span from K~/V rings kept across consecutive units; P from
+//                the forward's lse; dS (bf16); dQ~ += dS K~ in TMEM;
+//                epilogue: RoPE^T and the RMSNorm backward against the raw q,
+//                per-warp dw_q partials
 //   bwd_dkdv     key-stationary (M = 128 keys of one kv head): per 64-row
 //                query chunk (16 tokens x 4 heads) S^T = K~Q~^T and
-//                dP^T = V dA^T; P^T and dS^T (bf16, over S^T and dP^T);
+//                dP^T = V dA^T; P^T and dS^T (bf16, shared memory);
 //                dV += P^T dA and dK~ += dS^T Q~ in TMEM; epilogue: dv, and
 //                RoPE^T + RMSNorm backward against the raw k, dw_k partials
 //   dw_reduce    fixed-order sum of the weight-gradient partials
@@ -355,79 +354,6 @@ __device__ __forceinline__ void norm_rope_backward(uint32_t trow, float gscale, 
         dwacc[c] += warp_reduce_scatter32(pw);
     }
 }
-
-// ============================================================== dq kernel
-template <bool kSwa>
-struct DqCfg {
-    static constexpr int kN = kSwa ? 160 : 64;       // keys per tile (sliding window: the unit's span)
-    static constexpr int kNBuf = kSwa ? 1 : 2;       // S/dP buffers in TMEM
-    static constexpr int kStages = kSwa ? 2 : 4;     // K~/V stages in shared memory
-    static constexpr uint32_t kQHalf = 128 * kHalfRowBytes;   // 16 KiB
-    static constexpr uint32_t kQTile = 2 * kQHalf;
-    static constexpr uint32_t kKHalf = kN * kHalfRowBytes;
-    static constexpr uint32_t kKTile = 2 * kKHalf;
-    static constexpr uint32_t kOffQ = 0;
-    static constexpr uint32_t kOffA = kOffQ + kQTile;
-    static constexpr uint32_t kOffK = kOffA + kQTile;
-    static constexpr uint32_t kOffV = kOffK + kStages * kKTile;
-    static constexpr uint32_t kOffW = kOffV + kStages * kKTile;   // f32[128]
-    static constexpr uint32_t kOffBar = kOffW + 512;
-    static constexpr int kNumBars = 24;
-    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
-    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
-    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
-    static constexpr uint32_t kColDQ = kNBuf * 2 * kN;
-    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
-    static_assert(kColDQ + 128 <= 512, "TMEM budget");
-    // barrier indices
-    static constexpr int BQ_FULL = 0, BQ_EMPTY = 1, BKV_FULL = 2, BKV_EMPTY = BKV_FULL + kStages,
-                         BS_FULL = BKV_EMPTY + kStages, BDS_READY = BS_FULL + kNBuf,
-                         BS_FREE = BDS_READY + kNBuf, BACC_FULL = BS_FREE + kNBuf, BACC_FREE = BACC_FULL + 1,
-                         B_DRAIN = BACC_FREE + 1;
-    static_assert(B_DRAIN < kNumBars, "barrier count");
-};
-
-struct QUnit {
-    int b, kvh, qb, n;   // n: key tiles of the unit
-};
-
-template <bool kSwa>
-__device__ __forceinline__ bool dq_unit_at(const Params &p, int k, QUnit &x)
-{
-    const long long u = snake_unit(k);
-    if (u >= p.units) return false;
-    const long long per = (long long)p.B * p.Hkv;
-    x.qb = p.nq - 1 - (int)(u / per);
-    const long long strip = u % per;
-    x.b = (int)(strip / p.Hkv);
-    x.kvh = (int)(strip % p.Hkv);
-    x.n = kSwa ? 1 : min(p.nkt, (32 * x.qb + 31) / DqCfg<kSwa>::kN + 1);
-    return true;
-}
-
-// first key of tile j of a unit
-template <bool kSwa>
-__device__ __forceinline__ int dq_tile_key0(const QUnit &x, int j)
-{
-    return kSwa ? 32 * x.qb - 128 : j * DqCfg<kSwa>::kN;
-}
-
-template <bool kSwa>
-struct DqWalk {
-    int k = 0, j = 0;
-    QUnit x;
-    bool valid = false;
-    __device__ __forceinline__ void init(const Params &p) { k = 0; j = 0; valid = dq_unit_at<kSwa>(p, 0, x); }
-    __device__ __forceinline__ bool last() const { return j == x.n - 1; }
-    __device__ __forceinline__ void next(const Params &p)
-    {
-        if (++j == x.n) {
-            j = 0;
-            ++k;
-            valid = dq_unit_at<kSwa>(p, k, x);
-        }
-    }
-};
 
 // ====================================================== dq kernel, sliding window
 // Query-stationary: unit = 32 query tokens x 4 heads (M = 128 rows) of one
@@ -791,26 +717,6 @@ bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
 }
 
-// Row `row` of a swizzled two-half shared-memory tile (halves `hs` bytes
-// apart), 128 bf16, into 64 TMEM columns of this thread's lane from `taddr`
-// (bf16 pairs, the layout of a TMEM A operand).
-__device__ __forceinline__ void smem_row_to_tmem(uint32_t tile, uint32_t hs, int row, uint32_t taddr)
-{
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 v = lds128(tile + swa::chunk_off(row, 4 * q + c, hs));
-            w[4 * c] = v.x;
-            w[4 * c + 1] = v.y;
-            w[4 * c + 2] = v.z;
-            w[4 * c + 3] = v.w;
-        }
-        tmem_st16(taddr + 16 * q, w);
-    }
-}
-
 // Store 32 consecutive bf16 (16 packed words) as chunks c0 .. c0 + 3 of row
 // `row` of a single-half swizzled K-major tile (128-byte rows).
 __device__ __forceinline__ void sts_row_chunks(uint32_t tile, int row, int c0, const uint32_t (&w)[16])
@@ -819,273 +725,6 @@ __device__ __forceinline__ void sts_row_chunks(uint32_t tile, int row, int c0, c
     for (int q = 0; q < 4; ++q)
         sts128(tile + (uint32_t)row * kHalfRowBytes + ((uint32_t)((c0 + q) ^ (row & 7)) << 4),
                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
-}
-
-// ====================================================== dq kernel, full causal
-// Query-stationary (M = 128 rows = 4 heads x 32 tokens) over 64-key tiles.
-// The unit's Q~ and dA are copied once into TMEM, so S = Q~K~^T and
-// dP = dA V^T take their A operand from TMEM (two TMEM buffers).  Eight warps
-// (two per TMEM lane quarter, 32 of the 64 key columns each) load S and dP,
-// release the buffer, and write dS as bf16 into shared memory, from where
-// dQ~ += dS K~ reads it.  Warps 4-7 run the epilogue.
-struct DqFullCfg {
-    static constexpr int kN = 64;
-    static constexpr int kStages = 4;
-    static constexpr uint32_t kQHalf = 128 * kHalfRowBytes;
-    static constexpr uint32_t kQTile = 2 * kQHalf;
-    static constexpr uint32_t kKHalf = kN * kHalfRowBytes;
-    static constexpr uint32_t kKTile = 2 * kKHalf;
-    static constexpr uint32_t kDSTile = 128 * kHalfRowBytes;   // dS: 128 rows x 64 keys bf16
-    static constexpr uint32_t kOffQ = 0;
-    static constexpr uint32_t kOffA = kOffQ + kQTile;
-    static constexpr uint32_t kOffK = kOffA + kQTile;
-    static constexpr uint32_t kOffV = kOffK + kStages * kKTile;
-    static constexpr uint32_t kOffDS = kOffV + kStages * kKTile;
-    static constexpr uint32_t kOffW = kOffDS + kDSTile;
-    static constexpr uint32_t kOffBar = kOffW + 512;
-    static constexpr int kNumBars = 24;
-    static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
-    static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
-    static constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
-    // TMEM columns: Q~, dA (A operands), two {S, dP} buffers, dQ~
-    static constexpr uint32_t kColQ = 0, kColA = 64, kColBuf = 128, kBufStride = 128, kColDQ = 384;
-    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
-    static constexpr int BQ_FULL = 0, BQ_EMPTY = 1, BSTAT = 2, BKV_FULL = 3, BKV_EMPTY = BKV_FULL + kStages,
-                         BS_FULL = BKV_EMPTY + kStages, BS_FREE = BS_FULL + 2, BDS_READY = BS_FREE + 2,
-                         BDS_FREE = BDS_READY + 1, BACC_FULL = BDS_FREE + 1, BACC_FREE = BACC_FULL + 1,
-                         B_DRAIN = BACC_FREE + 1;
-    static_assert(B_DRAIN < kNumBars, "barrier count");
-};
-
-static_assert(DqFullCfg::kN == DqCfg<false>::kN, "full-causal dq units are walked with the 64-key tiling");
-
-template <int R>
-__global__ void __launch_bounds__(kThreads, 1)
-bwd_dq_full_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
-                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ Params p)
-{
-    using C = DqFullCfg;
-    constexpr int kN = C::kN, kStages = C::kStages;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(smem);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
-    Abort ab{reinterpret_cast<volatile int *>(smem + C::kOffAbort)};
-    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * (uint32_t)i; };
-    const int nunits = snake_count(p.units);
-
-    if (tid == 0) {
-        *ab.flag = 0;
-        mbar_init(bar(C::BQ_FULL), 1);
-        mbar_init(bar(C::BQ_EMPTY), 8);
-        mbar_init(bar(C::BSTAT), 8);
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(bar(C::BKV_FULL + i), 1);
-            mbar_init(bar(C::BKV_EMPTY + i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bar(C::BS_FULL + i), 1);
-            mbar_init(bar(C::BS_FREE + i), 8);
-        }
-        mbar_init(bar(C::BDS_READY), 8);
-        mbar_init(bar(C::BDS_FREE), 1);
-        mbar_init(bar(C::BACC_FULL), 1);
-        mbar_init(bar(C::BACC_FREE), 4);
-        mbar_init(bar(C::B_DRAIN), 1);
-        fence_barrier_init();
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_a);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-    }
-    if (tid < 128) reinterpret_cast<float *>(smem + C::kOffW)[tid] = __bfloat162float(p.w[tid]);
-    if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ================================================= TMA producer
-        if (lane == 0) {
-            int g = 0, k = 0;
-            QUnit x;
-            bool ok = true;
-            for (; k < nunits && ok; ++k) {
-                dq_unit_at<false>(p, k, x);
-                ok = mbar_wait(bar(C::BQ_EMPTY), (k & 1) ^ 1u, ab);
-                if (!ok) break;
-                mbar_arrive_expect_tx(bar(C::BQ_FULL), 2 * C::kQTile);
-                for (int h = 0; h < 2; ++h) {
-                    tma_load_4d(sbase + C::kOffQ + h * C::kQHalf, &tm_q, bar(C::BQ_FULL), h * 64, x.kvh * 4,
-                                x.qb * 32, x.b);
-                    tma_load_4d(sbase + C::kOffA + h * C::kQHalf, &tm_a, bar(C::BQ_FULL), h * 64, x.kvh * 4,
-                                x.qb * 32, x.b);
-                }
-                for (int j = 0; j < x.n && ok; ++j, ++g) {
-                    const int st = g % kStages;
-                    ok = mbar_wait(bar(C::BKV_EMPTY + st), ((g / kStages) & 1) ^ 1u, ab);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(bar(C::BKV_FULL + st), 2 * C::kKTile);
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_4d(sbase + C::kOffK + st * C::kKTile + h * C::kKHalf, &tm_k,
-                                    bar(C::BKV_FULL + st), h * 64, x.kvh, j * kN, x.b);
-                        tma_load_4d(sbase + C::kOffV + st * C::kKTile + h * C::kKHalf, &tm_v,
-                                    bar(C::BKV_FULL + st), h * 64, x.kvh, j * kN, x.b);
-                    }
-                }
-            }
-            for (int i = (g > kStages ? g - kStages : 0); i < g; ++i)
-                drain_wait(bar(C::BKV_FULL + i % kStages), (i / kStages) & 1);
-            if (k > 0) drain_wait(bar(C::BQ_FULL), (k - 1) & 1);
-        }
-    } else if (warp == 1) {
-        // ================================================= MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(128, kN, 0, 0);
-            const uint32_t idesc_dq = idesc_bf16_f32(128, 128, 0, 1);
-            DqWalk<false> ws, wd;
-            ws.init(p);
-            wd.init(p);
-            int ns = 0, nd = 0;
-            PollWatch watch;
-            while (wd.valid) {
-                bool progressed = false;
-                if (ws.valid && ns < nd + 2 && mbar_test(bar(C::BSTAT), ws.k & 1) &&
-                    mbar_test(bar(C::BKV_FULL + ns % kStages), (ns / kStages) & 1) &&
-                    mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
-                    tc_fence_after();
-                    const uint32_t dS = tmem + C::kColBuf + (ns & 1) * C::kBufStride;
-                    const uint32_t ks = sbase + C::kOffK + (ns % kStages) * C::kKTile;
-                    const uint32_t vs = sbase + C::kOffV + (ns % kStages) * C::kKTile;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
-                        mma_ts(dS, tmem + C::kColQ + kk * 8, smem_desc_sw128(ks + ok_, 16, 1024), idesc_s, kk > 0);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
-                        mma_ts(dS + kN, tmem + C::kColA + kk * 8, smem_desc_sw128(vs + ok_, 16, 1024), idesc_s,
-                               kk > 0);
-                    }
-                    mma_commit(bar(C::BS_FULL + (ns & 1)));
-                    ws.next(p);
-                    ++ns;
-                    progressed = true;
-                }
-                if (nd < ns && mbar_test(bar(C::BDS_READY), nd & 1) &&
-                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
-                    tc_fence_after();
-                    const uint32_t ks = sbase + C::kOffK + (nd % kStages) * C::kKTile;
-#pragma unroll
-                    for (int kk = 0; kk < kN / 16; ++kk)
-                        mma_ss(tmem + C::kColDQ, smem_desc_sw128(sbase + C::kOffDS + kk * 32, 16, 1024),
-                               smem_desc_sw128(ks + kk * 16 * 128, C::kKHalf, 1024), idesc_dq, (wd.j > 0 || kk > 0));
-                    mma_commit(bar(C::BKV_EMPTY + nd % kStages));
-                    mma_commit(bar(C::BDS_FREE));
-                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
-                    wd.next(p);
-                    ++nd;
-                    progressed = true;
-                }
-                if (!watch.tick(progressed, ab)) break;
-            }
-            mma_commit(bar(C::B_DRAIN));
-            drain_wait(bar(C::B_DRAIN), 0);
-        }
-        __syncwarp();
-    } else if (warp >= 4) {
-        // ================================================= Q~/dA into TMEM; dS (8 warps); epilogue (warps 4-7)
-        const int grp = (warp - 4) >> 2;           // key-column half of each tile
-        const int r = 32 * (warp & 3) + lane;      // query row (TMEM lane)
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
-        float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
-        bool ok = true;
-        int g = 0;
-        QUnit x;
-        for (int k = 0; k < nunits && ok; ++k) {
-            dq_unit_at<false>(p, k, x);
-            // every MMA reading the previous unit's Q~/dA has completed: this warp
-            // consumed the S/dP of that unit's last tile
-            ok = warp_wait(bar(C::BQ_FULL), k & 1, ab);
-            if (!ok) break;
-            if (grp == 0)
-                smem_row_to_tmem(sbase + C::kOffQ, C::kQHalf, r, tmem + lane_base + C::kColQ);
-            else
-                smem_row_to_tmem(sbase + C::kOffA, C::kQHalf, r, tmem + lane_base + C::kColA);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(C::BSTAT));
-                mbar_arrive(bar(C::BQ_EMPTY));
-            }
-            const int i = x.qb * 32 + (r >> 2);
-            const float2 rec = p.ld[(((long long)x.b * p.Hkv + x.kvh) * p.Tp + x.qb * 32) * 4 + r];
-            const float lse2 = rec.x, Dv = rec.y;
-            for (int j = 0; j < x.n && ok; ++j, ++g) {
-                const int bb = g & 1;
-                ok = warp_wait(bar(C::BS_FULL + bb), (g >> 1) & 1, ab);
-                if (!ok) break;
-                tc_fence_after();
-                uint32_t s[32], d[32], pk[16];
-                const uint32_t ts = tmem + lane_base + C::kColBuf + bb * C::kBufStride + 32 * grp;
-                tmem_ld32(ts, s);
-                tmem_ld32(ts + kN, d);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::BS_FREE + bb));   // the scores are in registers
-                const int hi = i - j * kN - 32 * grp;                // visible columns e <= hi
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p0 = ex2(fmaf(__uint_as_float(s[e]), p.sl2, -lse2));
-                    float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), p.sl2, -lse2));
-                    p0 = (e <= hi) ? p0 : 0.f;
-                    p1 = (e + 1 <= hi) ? p1 : 0.f;
-                    pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(d[e]) - Dv), p1 * (__uint_as_float(d[e + 1]) - Dv));
-                }
-                // the previous tile's dQ MMA has read the dS tile
-                ok = warp_wait(bar(C::BDS_FREE), (g & 1) ^ 1u, ab);
-                if (!ok) break;
-                sts_row_chunks(sbase + C::kOffDS, r, 4 * grp, pk);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::BDS_READY));
-            }
-            if (!ok || grp != 0) continue;
-            // ---- epilogue of the unit (warps 4-7): dq, dw_q
-            ok = warp_wait(bar(C::BACC_FULL), k & 1, ab);
-            if (!ok) break;
-            tc_fence_after();
-            const bool valid = i < p.T;
-            const long long off = valid ? (((long long)x.b * p.T + i) * p.Hq + x.kvh * 4 + (r & 3)) * kD : 0;
-            norm_rope_backward<R>(tmem + lane_base + C::kColDQ, p.scale, p.x + off, valid, w, p.eps, i, p.theta,
-                                  p.dx + off, dwacc);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::BACC_FREE));
-        }
-        if (grp == 0) {
-            float *dst = p.dw_part + ((long long)blockIdx.x * 4 + (warp & 3)) * kD;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
 }
 
 // ============================================================ dk/dv kernel

@@ -18,6 +18,7 @@
 #include "full_fwd.cuh"
 #include "decode.cuh"
 #include "bwd.cuh"
+#include "bwd_full.cuh"
 
 namespace {
 
@@ -50,9 +51,8 @@ bool set_bwd_smem()
 {
     using namespace gswa::bwd;
     return set_smem(bwd_dq_swa_kernel<R>, DqSwaCfg::kSmemBytes) ||
-           set_smem(bwd_dq_full_kernel<R>, DqFullCfg::kSmemBytes) ||
            set_smem(bwd_dkdv_kernel<R, true>, KvCfg::kSmemBytes) ||
-           set_smem(bwd_dkdv_kernel<R, false>, KvCfg::kSmemBytes);
+           set_smem(gswa::bwdf::bwd_full_kernel<R>, gswa::bwdf::kSmemBytes);
 }
 
 // Rotated dims the kernels are compiled for (the row is held in registers).
@@ -115,6 +115,20 @@ int encode_bthd(CUtensorMap *m, const void *base, int B, int T, int H, int D, in
                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
+}
+
+// 4-D f32 tensor map over [B, T, H, D] with a {32, box_h, box_t, 1} box (one
+// 128-byte swizzled row of 32 floats per (token, head)), for reduce-adds.
+int encode_bthd_f32(CUtensorMap *m, const void *base, int B, int T, int H, int D, int box_h, int box_t)
+{
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+    cuuint32_t box[4] = {32, (cuuint32_t)box_h, (cuuint32_t)box_t, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
 }
 
@@ -283,36 +297,152 @@ BwdWs bwd_ws_layout(const gswa_shape_t *s, bool gated)
     return w;
 }
 
+// Full-causal backward workspace: prepared q~ [B,T,Hq,D] and k~ [B,T,Hkv,D]
+// (bf16), the row records [B,Hkv,Tp,4] float2, the dq~ accumulator
+// [B,T,Hq,D] f32, the dw_q partials of the post kernel and the dw_k partials
+// of the fused kernel (f32 [n][128]).
+struct FullBwdWs {
+    size_t qt, kt, ld, acc, pq, pk, total;
+};
+
+FullBwdWs full_bwd_ws_layout(const gswa_shape_t *s)
+{
+    const size_t BT = (size_t)s->B * s->T;
+    const size_t Tp = ((size_t)s->T + 31) / 32 * 32;
+    FullBwdWs w;
+    w.qt = 0;
+    w.kt = w.qt + align256(BT * s->Hq * s->D * 2);
+    w.ld = w.kt + align256(BT * s->Hkv * s->D * 2);
+    w.acc = w.ld + align256((size_t)s->B * s->Hkv * Tp * 4 * 8);
+    w.pq = w.acc + align256(BT * s->Hq * s->D * 4);
+    w.pk = w.pq + align256((size_t)gswa::bwdf::kPostMaxGrid * gswa::bwdf::kPostWarps * 128 * 4);
+    w.total = w.pk + align256((size_t)gswa::bwdf::kMaxGrid * 4 * 128 * 4);
+    return w;
+}
+
 struct BwdMaps {
     CUtensorMap tq, ta, tk, tv;       // dq kernel
     CUtensorMap tk2, tv2, tq2, ta2;   // dk/dv kernel
 };
 
-template <int R, bool kSwa>
-void launch_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::bwd::Params &pk, unsigned gq,
-                     unsigned gk, cudaStream_t st)
+// The gated sliding-window backward's two main kernels.
+template <int R>
+void launch_swa_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::bwd::Params &pk, unsigned gq,
+                         unsigned gk, cudaStream_t st)
 {
     using namespace gswa::bwd;
-    if constexpr (kSwa)
-        bwd_dq_swa_kernel<R><<<gq, kThreads, DqSwaCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
-    else
-        bwd_dq_full_kernel<R><<<gq, kThreads, DqFullCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
-    bwd_dkdv_kernel<R, kSwa><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
+    bwd_dq_swa_kernel<R><<<gq, kThreads, DqSwaCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
+    bwd_dkdv_kernel<R, true><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
 }
 
-template <bool kSwa>
-void dispatch_bwd_main(int R, const BwdMaps &m, const gswa::bwd::Params &pq, const gswa::bwd::Params &pk,
-                       unsigned gq, unsigned gk, cudaStream_t st)
+template <int R>
+void launch_full_bwd(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tq, const CUtensorMap &ta,
+                     const CUtensorMap &tdq, const gswa::bwdf::Params &p, unsigned grid,
+                     const gswa::bwdf::PostParams &pp, unsigned pgrid, cudaStream_t st)
 {
-    switch (R) {
-    case 0: launch_bwd_main<0, kSwa>(m, pq, pk, gq, gk, st); break;
-    case 42: launch_bwd_main<42, kSwa>(m, pq, pk, gq, gk, st); break;
-    case 64: launch_bwd_main<64, kSwa>(m, pq, pk, gq, gk, st); break;
-    default: launch_bwd_main<128, kSwa>(m, pq, pk, gq, gk, st); break;
-    }
+    using namespace gswa::bwdf;
+    bwd_full_kernel<R><<<grid, kThreads, kSmemBytes, st>>>(tk, tv, tq, ta, tdq, p);
+    bwd_dq_post_kernel<R><<<pgrid, kPostWarps * 32, 0, st>>>(pp);
 }
 
-// Shared body of gswa_bwd (swa: gated sliding window) and full_attn_bwd.
+// full_attn_bwd after the argument checks: records, q~/k~, the fused
+// key-stationary kernel (dk, dv, dw_k partials, dq~ sums), the dq post pass
+// and the fixed-order weight-gradient sums.
+int run_full_bwd(const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *w_q,
+                 const void *w_k, const void *y, const float *lse, const void *dy, void *dq, void *dk, void *dv,
+                 float *dw_q, float *dw_k, void *workspace, int num_sms, cudaStream_t st)
+{
+    const FullBwdWs L = full_bwd_ws_layout(s);
+    char *ws = static_cast<char *>(workspace);
+    void *qt = ws + L.qt, *kt = ws + L.kt, *acc = ws + L.acc;
+    float2 *ld = reinterpret_cast<float2 *>(ws + L.ld);
+    float *part_q = reinterpret_cast<float *>(ws + L.pq), *part_k = reinterpret_cast<float *>(ws + L.pk);
+    const int Tp = (s->T + 31) / 32 * 32;
+
+    // 1. row records {lse log2 e, D = sum dy y}
+    gswa::bwd::PrepParams pp;
+    std::memset(&pp, 0, sizeof pp);
+    pp.y = static_cast<const __nv_bfloat16 *>(y);
+    pp.dy = static_cast<const __nv_bfloat16 *>(dy);
+    pp.lse = lse;
+    pp.ld = ld;
+    pp.rows = (long long)s->B * Tp * s->Hq;
+    pp.T = s->T;
+    pp.Tp = Tp;
+    pp.Hq = s->Hq;
+    long long pgrid = ((long long)s->B * Tp + 15) / 16;
+    if (pgrid > 16LL * num_sms) pgrid = 16LL * num_sms;
+    gswa::bwd::bwd_prep_kernel<<<(unsigned)pgrid, 256, 0, st>>>(pp);
+    // 2. prepared queries and keys; 3. the dq~ accumulator starts at zero
+    int rc = launch_qk_prep(s, s->Hq, q, w_q, qt, 0, st, num_sms);
+    if (rc == GSWA_OK) rc = launch_qk_prep(s, s->Hkv, k, w_k, kt, 0, st, num_sms);
+    if (rc != GSWA_OK) return rc;
+    if (cudaMemsetAsync(acc, 0, (size_t)s->B * s->T * s->Hq * s->D * 4, st) != cudaSuccess) return GSWA_ERR_LAUNCH;
+
+    // 4. the fused kernel
+    using namespace gswa::bwdf;
+    CUtensorMap tk, tv, tq, ta, tdq;
+    if (encode_bthd(&tk, kt, s->B, s->T, s->Hkv, s->D, 1, kKeys) ||
+        encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, kKeys) ||
+        encode_bthd(&tq, qt, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
+        encode_bthd(&ta, dy, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
+        encode_bthd_f32(&tdq, acc, s->B, s->T, s->Hq, s->D, 4, kChTok))
+        return GSWA_ERR_INVALID_ARG;
+    Params p;
+    std::memset(&p, 0, sizeof p);
+    p.B = s->B;
+    p.T = s->T;
+    p.Tp = Tp;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.nkt = (s->T + kKeys - 1) / kKeys;
+    p.units = (long long)s->B * s->Hkv * p.nkt;
+    p.eps = s->eps;
+    p.scale = s->scale;
+    p.sl2 = s->scale * 1.4426950408889634f;
+    p.ld = ld;
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.dw_part = part_k;
+    fill_theta(p.theta, s->rope_dims, s->rope_base);
+    long long grid = p.units < num_sms ? p.units : num_sms;
+    if (grid > kMaxGrid) grid = kMaxGrid;
+
+    // 5. dq from the accumulated dq~
+    PostParams q2;
+    std::memset(&q2, 0, sizeof q2);
+    q2.acc = static_cast<const float *>(acc);
+    q2.q = static_cast<const __nv_bfloat16 *>(q);
+    q2.wq = static_cast<const __nv_bfloat16 *>(w_q);
+    q2.dq = static_cast<__nv_bfloat16 *>(dq);
+    q2.dw_part = part_q;
+    q2.rows = (long long)s->B * s->T * s->Hq;
+    q2.T = s->T;
+    q2.Hq = s->Hq;
+    q2.eps = s->eps;
+    q2.scale = s->scale;
+    fill_theta(q2.theta, s->rope_dims, s->rope_base);
+    long long qgrid = (q2.rows / kPostRows + kPostWarps - 1) / kPostWarps;
+    if (qgrid > 3LL * num_sms) qgrid = 3LL * num_sms;
+    if (qgrid > kPostMaxGrid) qgrid = kPostMaxGrid;
+
+    switch (s->rope_dims) {
+    case 0: launch_full_bwd<0>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    case 42: launch_full_bwd<42>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    case 64: launch_full_bwd<64>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    default: launch_full_bwd<128>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    }
+    // 6. weight gradients, summed in a fixed order
+    const unsigned rt = gswa::bwd::kD * gswa::bwd::kReduceSlices;
+    gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_q, (int)qgrid * kPostWarps, dw_q);
+    gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_k, (int)grid * 4, dw_k);
+    return cudaGetLastError() == cudaSuccess ? GSWA_OK : GSWA_ERR_LAUNCH;
+}
+
+// Shared argument checks of gswa_bwd (swa: gated sliding window) and
+// full_attn_bwd, then the gated path here or the full-causal one in run_full_bwd.
 int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const void *v, const void *g,
             const void *w_q, const void *w_k, const void *y, const float *lse, const void *dy, void *dq,
             void *dk, void *dv, void *dg, float *dw_q, float *dw_k, void *workspace, size_t workspace_bytes,
@@ -341,11 +471,14 @@ int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const
         !aligned16(dk) || !aligned16(dv) || (swa && (!aligned16(g) || !aligned16(dg))) ||
         (reinterpret_cast<uintptr_t>(lse) & 3u))
         return GSWA_ERR_MISALIGNED;
-    const BwdWs L = bwd_ws_layout(s, swa);
-    if (workspace == nullptr || workspace_bytes < L.total) return GSWA_ERR_WORKSPACE_TOO_SMALL;
+    const size_t need = swa ? bwd_ws_layout(s, true).total : full_bwd_ws_layout(s).total;
+    if (workspace == nullptr || workspace_bytes < need) return GSWA_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return GSWA_ERR_MISALIGNED;
     rc = device_setup(&num_sms);
     if (rc != GSWA_OK) return rc;
+    if (!swa)
+        return run_full_bwd(s, q, k, v, w_q, w_k, y, lse, dy, dq, dk, dv, dw_q, dw_k, workspace, num_sms, st);
+    const BwdWs L = bwd_ws_layout(s, swa);
 
     char *ws = static_cast<char *>(workspace);
     void *qt = ws + L.qt, *kt = ws + L.kt;
@@ -375,9 +508,8 @@ int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const
     if (rc == GSWA_OK) rc = launch_qk_prep(s, s->Hkv, k, w_k, kt, 0, st, num_sms);
     if (rc != GSWA_OK) return rc;
 
-    // 3. dq and dk/dv
-    // dq kernel's K~/V boxes: 32-key ring blocks (sliding window), 64-key tiles (full causal)
-    const int kN = swa ? gswa::bwd::DqSwaCfg::kTok : gswa::bwd::DqCfg<false>::kN;
+    // 3. dq and dk/dv (the dq kernel's K~/V boxes are its 32-key ring blocks)
+    const int kN = gswa::bwd::DqSwaCfg::kTok;
     BwdMaps m;
     if (encode_bthd(&m.tq, qt, s->B, s->T, s->Hq, s->D, 4, 32) ||
         encode_bthd(&m.ta, da, s->B, s->T, s->Hq, s->D, 4, 32) ||
@@ -426,10 +558,12 @@ int run_bwd(bool swa, const gswa_shape_t *s, const void *q, const void *k, const
         return (unsigned)(gsz < gswa::bwd::kMaxGrid ? gsz : gswa::bwd::kMaxGrid);
     };
     const unsigned gq = grid_of(pq.units), gk = grid_of(pk.units);
-    if (swa)
-        dispatch_bwd_main<true>(s->rope_dims, m, pq, pk, gq, gk, st);
-    else
-        dispatch_bwd_main<false>(s->rope_dims, m, pq, pk, gq, gk, st);
+    switch (s->rope_dims) {
+    case 0: launch_swa_bwd_main<0>(m, pq, pk, gq, gk, st); break;
+    case 42: launch_swa_bwd_main<42>(m, pq, pk, gq, gk, st); break;
+    case 64: launch_swa_bwd_main<64>(m, pq, pk, gq, gk, st); break;
+    default: launch_swa_bwd_main<128>(m, pq, pk, gq, gk, st); break;
+    }
     // 4. weight gradients, summed in a fixed order
     const unsigned rt = gswa::bwd::kD * gswa::bwd::kReduceSlices;
     gswa::bwd::dw_reduce_kernel<<<1, rt, 0, st>>>(part_q, (int)gq * 4, dw_q);
@@ -592,9 +726,9 @@ int full_attn_fwd(const gswa_shape_t *s, const void *q, const void *k, const voi
     p.T = s->T;
     p.Hq = s->Hq;
     p.Hkv = s->Hkv;
-    p.nq = (s->T + gswa::full::kTok - 1) / gswa::full::kTok;
+    p.nm = (s->T + gswa::full::kUnitTok - 1) / gswa::full::kUnitTok;
     p.nkt = (s->T + gswa::full::kKeys - 1) / gswa::full::kKeys;
-    p.units = (long long)s->B * s->Hkv * p.nq;
+    p.units = (long long)s->B * s->Hkv * p.nm;
     p.sl2 = s->scale * 1.4426950408889634f;
     p.wq = static_cast<const __nv_bfloat16 *>(w_q);
     p.wk = static_cast<const __nv_bfloat16 *>(w_k);
@@ -723,7 +857,7 @@ size_t gswa_workspace_bytes(int op, const gswa_shape_t *s)
     case GSWA_OP_GSWA_FWD: return swa_fwd_ws(s);
     case GSWA_OP_FULL_FWD: return full_fwd_ws(s);
     case GSWA_OP_GSWA_BWD: return bwd_ws_layout(s, true).total;
-    case GSWA_OP_FULL_BWD: return bwd_ws_layout(s, false).total;
+    case GSWA_OP_FULL_BWD: return full_bwd_ws_layout(s).total;
     case GSWA_OP_FULL_DECODE: return s->cache_len > 0 ? full_decode_ws(s) : 0;
     default: return 0;
     }

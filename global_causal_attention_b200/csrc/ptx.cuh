@@ -117,13 +117,20 @@ struct Abort {
 // false (and raises the CTA's abort flag) when the wait gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort &ab)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    // fast path: a non-blocking test (a blocking try_wait could sit out a
+    // lowered limit inside the hardware's own suspend window)
+    if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    // a lowered limit (below 1 ms) is checked on every pass, with a suspend hint
+    // no longer than the limit itself
+    const unsigned long long lim = g_wait_limit_ns;
+    const bool eager = lim < 1000000ull;
+    const uint32_t hint = eager ? (uint32_t)lim : 1000000u;
     for (uint32_t spin = 0;; ++spin) {
-        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-        if ((spin & 3u) == 3u) {
+        if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+        if (eager || (spin & 3u) == 3u) {
             if (ab.raised()) return false;
-            if (globaltimer() - t0 > g_wait_limit_ns) {
+            if (globaltimer() - t0 > lim) {
                 ab.raise(kStatusTimeout);
                 return false;
             }
@@ -133,26 +140,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
 
 // Stall watchdog of a polling loop (a thread that tests several barriers in
 // turn): call tick(progressed) once per pass.  The wall clock is a slow read,
-// so it is consulted only every 512 idle passes.  Returns false (with the
-// CTA's abort flag raised) once the loop has made no progress for
-// g_wait_limit_ns, or when another role raised the flag.
+// so it is consulted only every 512 idle passes (every 8 under a lowered
+// limit).  Returns false (with the CTA's abort flag raised) once the loop has
+// made no progress for g_wait_limit_ns, or when another role raised the flag.
 struct PollWatch {
     uint32_t idle = 0;
     uint64_t t0 = 0;
+    unsigned long long lim = g_wait_limit_ns;
+    uint32_t mask = lim < 1000000ull ? 7u : 511u;
     __device__ __forceinline__ bool tick(bool progressed, const Abort &ab)
     {
         if (progressed) {
             idle = 0;
             return true;
         }
-        if ((++idle & 511u) != 0) return true;
+        if ((++idle & mask) != 0) return true;
         if (ab.raised()) return false;
         const uint64_t now = globaltimer();
-        if (idle == 512u) {
+        if (idle == mask + 1) {
             t0 = now;
             return true;
         }
-        if (now - t0 > g_wait_limit_ns) {
+        if (now - t0 > lim) {
             ab.raise(kStatusTimeout);
             return false;
         }
@@ -218,6 +227,23 @@ __device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src, int
             reinterpret_cast<uint64_t>(tmap)),
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
+}
+
+// Element-wise add of a shared-memory tile into global memory through a tensor
+// map (the tensor map's element type, here f32); the adds of different CTAs
+// to the same elements are atomic, their order unspecified.
+__device__ __forceinline__ void tma_reduce_add_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a
@@ -399,27 +425,21 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// Hardware tanh approximation (one MUFU op, |relative error| < 2^-10.9).
-__device__ __forceinline__ float tanh_approx(float x)
-{
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// σ(x) = (1 + tanh(x/2)) / 2 of a packed bf16 pair, evaluated on f16 pairs
-// (one MUFU op per pair); returns the packed f16 pair.  A bf16 value is exact
-// in f16 over f16's normal range; outside it the f16 rounding only moves x
-// where σ is already flat (|x| > 65504 gives 0 or 1, tiny |x| gives 1/2).
+// σ(x) = (1 + tanh(x/2)) / 2 in f32 (one hardware tanh per element, relative
+// error below 2^-10.9) of a packed bf16 pair, returned as a packed f16 pair
+// (lo in the low half): the gate tile holds σ in place of g, two bytes per
+// element, and f16 keeps 11 significant bits where bf16 would keep 8.  On
+// one B200 this matched 1 / (1 + 2^(-x log2 e)) (hardware 2^x and reciprocal)
+// in the output error, at the cost of the f16 tanh form, 13 % below it.
 __device__ __forceinline__ uint32_t sigmoid_bf16x2_f16x2(uint32_t g)
 {
-    const uint32_t half2 = 0x38003800u;   // {0.5, 0.5} in f16
-    uint32_t h, t, s;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(__uint_as_float(g & 0xFFFF0000u)), "f"(__uint_as_float(g << 16)));
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(h), "r"(half2));
-    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
-    asm("fma.rn.f16x2 %0, %1, %2, %2;" : "=r"(s) : "r"(t), "r"(half2));
-    return s;
+    const float lo = __uint_as_float(g << 16), hi = __uint_as_float(g & 0xFFFF0000u);
+    float tl, th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tl) : "f"(0.5f * lo));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(0.5f * hi));
+    uint32_t h;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(fmaf(0.5f, th, 0.5f)), "f"(fmaf(0.5f, tl, 0.5f)));
+    return h;
 }
 
 // Packed f32 pairs: sm_100 executes add/mul/fma on .f32x2 operands as two

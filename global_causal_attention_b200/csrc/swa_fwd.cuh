@@ -31,7 +31,7 @@
 // next K block's load never waits behind a softmax.
 //   warps 4-7   query prologue: RMSNorm + RoPE of the 128 Q rows, in place
 //   warps 8-11  softmax: S (TMEM) -> P (bf16, TMEM), 1/l (TMEM), lse
-//   warps 12-15 epilogue: σ(g) into the gate tile ahead of time, then
+//   warps 12-15 epilogue: σ(g) (f32, stored as f16) into the gate tile ahead of time, then
 //               O (TMEM) * 1/l * σ -> y in the gate tile, TMA store; its thread 0
 //               also loads the gate tiles (2 stages), reusing each slot as soon
 //               as the y store has read it
@@ -728,7 +728,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         };
         if (r == 0)
             while (g_issued < n && g_issued < 2) load_gate();
-        // σ(g) = (1 + tanh(g/2)) / 2 over this thread's row of gate tile `idx`
+        // σ(g) = (1 + tanh(g/2)) / 2 (f32, kept as f16) over this thread's row of gate tile `idx`
         auto sigma_row = [&](int idx) -> bool {
             if (!warp_wait(bar(BG_FULL + (idx & 1)), (idx >> 1) & 1, ab)) return false;
             const uint32_t ga = sbase + kOffG + (idx & 1) * kTileBytes;

@@ -133,6 +133,9 @@ int gswa_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void
  * §2.2 and §3.1 as for gswa_bwd).  The formulas of gswa_bwd with σ = 1
  * (dA = dy) over every key j <= i; no g, no dg.  Layouts, workspace
  * (gswa_workspace_bytes(GSWA_OP_FULL_BWD)) and ownership as for gswa_bwd.
+ * dk, dv and dw_k are bitwise reproducible; dq~ is summed in f32 by
+ * reduce-adds whose order across key tiles is not fixed, so dq and dw_q may
+ * differ between runs in their last bits.
  */
 int full_attn_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,
                   const void *w_q, const void *w_k, const void *y, const float *lse,

@@ -124,7 +124,10 @@ def test_workspace_sizes_follow_the_buffer_layouts(B, T, Hq, Hkv):
     assert gca.workspace_bytes(gca.OP_GSWA_FWD, s) == _a256(k)                      # k~
     assert gca.workspace_bytes(gca.OP_FULL_FWD, s) == _a256(k) + _a256(q)           # k~, q~
     assert gca.workspace_bytes(gca.OP_GSWA_BWD, s) == _a256(q) + _a256(k) + _a256(q) + _a256(rec) + 2 * part
-    assert gca.workspace_bytes(gca.OP_FULL_BWD, s) == _a256(q) + _a256(k) + _a256(rec) + 2 * part   # no dA
+    # full causal: q~, k~, records, the f32 dq~ accumulator, dw_q partials of the dq post pass
+    # (512 CTAs x 8 warps) and dw_k partials of the fused kernel (256 CTAs x 4 warps)
+    assert gca.workspace_bytes(gca.OP_FULL_BWD, s) == (_a256(q) + _a256(k) + _a256(rec) + _a256(2 * q)
+                                                        + _a256(512 * 8 * 128 * 4) + _a256(256 * 4 * 128 * 4))
     assert gca.workspace_bytes(gca.OP_GSWA_DECODE, s) == 0
 
 

@@ -90,11 +90,17 @@ def test_gate_precision_window_1():
     """With window 1 each row attends to its own key only (P = 1), so the
     kernel's output is bf16(v ⊙ σ~(g)) and its error against the exact
     v ⊙ σ(g) is the gate's evaluation error plus the final bf16 rounding.
-    The kernel evaluates σ on f16 pairs (one tanh.approx.f16x2 per pair);
-    this measures what that costs next to the unavoidable rounding of the
-    output to bf16, and bounds it."""
+    The kernel evaluates σ in f32 and keeps it as f16 until the product;
+    the error that adds, in quadrature on top of the unavoidable rounding of
+    the output to bf16, must stay well below that rounding."""
     s = Shape(B=2, T=2048, Hq=8, Hkv=2, window=1)
     x = attention_inputs(s, 21)
+    # one-dimension weight spikes select the exact row-max path, where the one
+    # visible score is its own maximum, so P = 2^0 = 1 and l = 1 exactly: no
+    # rounding of P enters the output, only the gate's and the output's
+    wq, wk = torch.ones(128), torch.ones(128)
+    wq[9], wk[100] = 4.0, 4.0
+    x["wq"], x["wk"] = wq.to(torch.bfloat16), wk.to(torch.bfloat16)
     y, _ = run_gpu(s, x)
     v = x["v"].double().repeat_interleave(4, dim=2)
     exact = v * torch.sigmoid(x["g"].double())
@@ -103,8 +109,8 @@ def test_gate_precision_window_1():
     nrm = exact.norm().item()
     e_gpu = (yd - exact).norm().item() / nrm
     e_round = (best - exact).norm().item() / nrm
-    e_gate = (yd - best).norm().item() / nrm
+    e_gate = max(e_gpu ** 2 - e_round ** 2, 0.0) ** 0.5
     print(f"gate precision: rel-L2 vs exact {e_gpu:.3e}; bf16 rounding alone {e_round:.3e}; "
-          f"gate evaluation {e_gate:.3e}; max |y - exact| {(yd - exact).abs().max().item():.3e}")
+          f"gate evaluation (in quadrature) {e_gate:.3e}; max |y - exact| {(yd - exact).abs().max().item():.3e}")
     assert e_gpu <= 5e-3
-    assert e_gate <= 2e-3
+    assert e_gate <= 0.5 * e_round

@@ -14,7 +14,7 @@ import pytest
 import global_causal_attention_b200 as gca
 import oracle
 from tests.parity import assert_fwd_close, assert_grad_close
-from workloads import WORKLOADS, attention_inputs
+from workloads import WORKLOADS, Shape, attention_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -40,17 +40,22 @@ def _run(op, s, xd):
 
 @pytest.mark.parametrize("op", ["gswa_fwd", "full_attn_fwd", "gswa_bwd", "full_attn_bwd"])
 def test_wait_that_runs_out_is_reported_and_the_next_call_is_clean(op):
-    s = WORKLOADS["tiny"]
-    x = attention_inputs(s, 40, with_grad=True)
-    xd = {n: t.cuda() for n, t in x.items()}
+    # the aborted call: a shape with many units per CTA, so that some waits
+    # (a producer whose ring is full, an epilogue waiting for a whole unit)
+    # last well past the 1 ns limit and the device timer's resolution
+    big = Shape(B=2, T=4096, Hq=8, Hkv=2)
+    xb = attention_inputs(big, 41, device="cuda", with_grad=True)
     assert gca.gswa_check_status() == 0
     gca.gswa_set_wait_limit_ns(1)
     try:
-        _run(op, s, xd)
+        _run(op, big, xb)
         rc = gca.gswa_check_status()
     finally:
         gca.gswa_set_wait_limit_ns(0)
     assert rc == TIMEOUT, f"{op}: status {rc} after a 1 ns wait limit"
+    s = WORKLOADS["tiny"]
+    x = attention_inputs(s, 40, with_grad=True)
+    xd = {n: t.cuda() for n, t in x.items()}
     # the default bound again: clean status, correct results
     out = _run(op, s, xd)
     assert gca.gswa_check_status() == 0
