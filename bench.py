@@ -58,8 +58,6 @@ LAUNCHES = {"gswa_fwd": 2, "gswa_bwd": 7, "full_attn_fwd": 3, "full_attn_bwd": 7
 # call's kernels).  Absent entries are reported as null: not captured for the
 # current kernels.
 TRAFFIC = {
-    ("train_4k", "full_attn_bwd"): 9_568_000_000,    # 8.96 GB read + 0.61 GB written, 7 launches
-    ("train_4k", "gswa_fwd"): 1_003_600_000,         # qk_prep 83.9 MB + attention 919.7 MB, 2 launches
     ("decode_256k", "full_decode"): 34_430_000_000,  # 34.40 GB read + 0.03 GB written, 3 launches
 }
 

@@ -56,28 +56,33 @@ constexpr int kThreads = 512;
 constexpr int kKeys = 128;                  // keys per unit (MMA M)
 constexpr int kChTok = 16;                  // tokens per query chunk
 constexpr int kChRows = 4 * kChTok;         // 64 query rows per chunk (MMA N of the score products)
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kMaxGrid = 256;               // CTAs (dw_k partials sizing)
 
 constexpr uint32_t kKHalf = kKeys * kHalfRowBytes;        // 16 KiB: 128 keys x 64 dims
 constexpr uint32_t kKTile = 2 * kKHalf;                   // 32 KiB
 constexpr uint32_t kCHalf = kChRows * kHalfRowBytes;      // 8 KiB: 64 rows x 64 dims
 constexpr uint32_t kCTile = 2 * kCHalf;                   // 16 KiB
+constexpr uint32_t kStageBytes = 2 * kCTile;              // Q~ and dA of one chunk
 constexpr uint32_t kRecBytes = kChRows * 8;               // {lse log2 e, D} per row
-constexpr uint32_t kStageBytes = 2 * kCTile + 1024;       // Q~, dA, records (keeps 1 KiB alignment)
 constexpr uint32_t kDSTile = kKeys * kHalfRowBytes;       // dS^T: 128 keys x 64 rows bf16
-constexpr uint32_t kStgBytes = kChRows * 128;             // 64 rows x 32 dims f32: one reduce box
+constexpr int kStgRows = 32;                              // rows of one reduce box (8 tokens x 4 heads)
+constexpr uint32_t kStgBytes = kStgRows * 128;            // 32 rows x 32 dims f32
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kKTile;
 constexpr uint32_t kOffSt = kOffV + kKTile;
 constexpr uint32_t kOffDS = kOffSt + kStages * kStageBytes;
-constexpr uint32_t kOffStg = kOffDS + kDSTile;            // 4 staging tiles, one per TMEM lane quarter
-constexpr uint32_t kOffW = kOffStg + 4 * kStgBytes;       // f32[128] w_k
+constexpr uint32_t kOffStg = kOffDS + kDSTile;            // one staging box per TMEM lane quarter
+constexpr uint32_t kOffRec = kOffStg + 4 * kStgBytes;     // records of each stage
+constexpr uint32_t kOffW = kOffRec + kStages * kRecBytes; // f32[128] w_k
 constexpr uint32_t kOffBar = kOffW + 512;
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 26;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
-constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+// No alignment slack: the kernel checks that the dynamic shared memory starts
+// on a 1 KiB boundary (it does, as the only allocation of a one-CTA-per-SM
+// kernel) and reports GSWA_ERR_LAUNCH through the status word otherwise.
+constexpr uint32_t kSmemBytes = kOffAbort + 4;
 static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
 static_assert((kOffSt % 1024) == 0 && (kStageBytes % 1024) == 0 && (kOffDS % 1024) == 0 && (kOffStg % 1024) == 0,
               "swizzled tiles are 1 KiB aligned");
@@ -155,14 +160,19 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
                 const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ Params p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
     const uint32_t sbase = smem_u32(smem);
+    if ((sbase & 1023u) != 0) {   // the swizzled tiles need 1 KiB alignment (uniform over the CTA)
+        if (threadIdx.x == 0) atomicExch(&g_status, kStatusSetup);
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
     Abort ab{reinterpret_cast<volatile int *>(smem + kOffAbort)};
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
     auto stage = [&](int st) -> uint32_t { return sbase + kOffSt + (uint32_t)st * kStageBytes; };
+    auto recs = [&](int st) -> uint32_t { return sbase + kOffRec + (uint32_t)st * kRecBytes; };
 
     if (tid == 0) {
         *ab.flag = 0;
@@ -232,7 +242,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     tma_load_4d(stage(st) + kCTile + h * kCHalf, &tm_a, bar(BST_FULL + st), h * 64, w.x.kvh * 4, t0,
                                 w.x.b);
                 }
-                bulk_load(stage(st) + 2 * kCTile, p.ld + (((long long)w.x.b * p.Hkv + w.x.kvh) * p.Tp + t0) * 4,
+                bulk_load(recs(st), p.ld + (((long long)w.x.b * p.Hkv + w.x.kvh) * p.Tp + t0) * 4,
                           kRecBytes, bar(BST_FULL + st));
             }
             // every copy this thread issued lands before shared memory is released
@@ -250,6 +260,14 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ws.init(p);
             wa.init(p);
             bool ok = true;
+            // shared-memory descriptors, built once: K-major (K~, V, dS^T, Q~ and dA of
+            // stage 0 as A/B of the score products and dK) and MN-major (K~ as the A of
+            // dQ^T; Q~, dA and dS^T as transposed B operands); the stages differ by a
+            // constant byte offset
+            const SmemDesc dK_k = make_desc(sbase + kOffK, 16, 1024), dV_k = make_desc(sbase + kOffV, 16, 1024);
+            const SmemDesc dK_mn = make_desc(sbase + kOffK, kKHalf, 1024);
+            const SmemDesc dS_k = make_desc(sbase + kOffDS, 16, 1024), dS_mn = make_desc(sbase + kOffDS, kDSTile, 1024);
+            const SmemDesc dC_k = make_desc(stage(0), 16, 1024), dC_mn = make_desc(stage(0), kCHalf, 1024);
             // S^T and dP^T of chunk ws.g
             auto issue_scores = [&]() -> bool {
                 const int g = ws.g;
@@ -259,22 +277,19 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 // the S buffer's previous P^T has been read by its dV
                 if (!mbar_wait(bar(BSB_FREE + (g & 1)), ((g >> 1) & 1) ^ 1u, ab)) return false;
                 tc_fence_after();
-                const uint32_t qs = stage(st), as = qs + kCTile;
+                const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;   // stage offsets
+                const uint32_t ds = tmem + kColS + (g & 1) * 64;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, co = (kk >> 2) * kCHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColS + (g & 1) * 64, smem_desc_sw128(sbase + kOffK + ko, 16, 1024),
-                           smem_desc_sw128(qs + co, 16, 1024), id_s, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(ds, dK_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
+                           dC_k.at(qo + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
                 // dP: the softmax warps have loaded the previous chunk's dP^T
                 if (!mbar_wait(bar(BDP_FREE), (g & 1) ^ 1u, ab)) return false;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * kKHalf + (kk & 3) * 32, co = (kk >> 2) * kCHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColDP, smem_desc_sw128(sbase + kOffV + ko, 16, 1024),
-                           smem_desc_sw128(as + co, 16, 1024), id_s, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + kColDP, dV_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
+                           dC_k.at(ao + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
                 mma_commit(bar(BS_FULL));
                 ws.next(p);
                 return true;
@@ -282,29 +297,29 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // dV, dK and dQ^T of chunk wa.g
             auto issue_acc = [&]() -> bool {
                 const int g = wa.g, st = g % kStages;
-                const uint32_t qs = stage(st), as = qs + kCTile;
+                const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;
                 if (!mbar_wait(bar(BP_READY + (g & 1)), (g >> 1) & 1, ab)) return false;
                 // the first chunk of a unit overwrites dV/dK: the previous unit's epilogue has read them
                 if (wa.j == 0 && !mbar_wait(bar(BACC_FREE), (wa.k & 1) ^ 1u, ab)) return false;
                 tc_fence_after();
                 const uint32_t pt = tmem + kColS + (g & 1) * 64;
+                const uint32_t acc0 = wa.j > 0;
 #pragma unroll
                 for (int kk = 0; kk < kChRows / 16; ++kk)
-                    mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8,
-                           smem_desc_sw128(as + kk * 16 * kHalfRowBytes, kCHalf, 1024), id_acc, (wa.j > 0 || kk > 0));
+                    mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8, dC_mn.at(ao + kk * 16 * kHalfRowBytes),
+                           id_acc, acc0 | (kk > 0));
                 mma_commit(bar(BSB_FREE + (g & 1)));
                 if (!mbar_wait(bar(BDS_READY), g & 1, ab)) return false;
                 if (!mbar_wait(bar(BDQ_FREE), (g & 1) ^ 1u, ab)) return false;
                 tc_fence_after();
-                const uint32_t ds = sbase + kOffDS;
 #pragma unroll
                 for (int kk = 0; kk < kChRows / 16; ++kk)
-                    mma_ss(tmem + kColDK, smem_desc_sw128(ds + kk * 32, 16, 1024),
-                           smem_desc_sw128(qs + kk * 16 * kHalfRowBytes, kCHalf, 1024), id_acc, (wa.j > 0 || kk > 0));
+                    mma_ss(tmem + kColDK, dS_k.at(kk * 32), dC_mn.at(qo + kk * 16 * kHalfRowBytes), id_acc,
+                           acc0 | (kk > 0));
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk)
-                    mma_ss(tmem + kColDQ, smem_desc_sw128(sbase + kOffK + kk * 16 * kHalfRowBytes, kKHalf, 1024),
-                           smem_desc_sw128(ds + kk * 16 * kHalfRowBytes, kDSTile, 1024), id_dq, kk > 0);
+                    mma_ss(tmem + kColDQ, dK_mn.at(kk * 16 * kHalfRowBytes), dS_mn.at(kk * 16 * kHalfRowBytes), id_dq,
+                           kk > 0);
                 mma_commit(bar(BDQ_FULL));
                 mma_commit(bar(BDS_FREE));
                 mma_commit(bar(BST_EMPTY + st));
@@ -317,13 +332,15 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             };
             if (ws.valid) ok = issue_scores();
             while (ok && wa.valid) {
-                // the next chunk's scores go ahead of this chunk's accumulation, except
-                // across a unit boundary (the next unit's K~/V load waits for this
-                // unit's last products)
+                // the next chunk's scores go ahead of this chunk's accumulation (so that
+                // its softmax overlaps these products) when its stage has landed;
+                // otherwise, and across a unit boundary (the next unit's K~/V load
+                // waits for this unit's last products), the accumulation goes first
                 const bool same_unit = ws.valid && ws.k == wa.k;
-                if (same_unit) ok = issue_scores();
+                const bool ready = same_unit && mbar_test(bar(BST_FULL + ws.g % kStages), (ws.g / kStages) & 1);
+                if (ready) ok = issue_scores();
                 if (ok) ok = issue_acc();
-                if (ok && !same_unit && ws.valid) ok = issue_scores();
+                if (ok && !ready && ws.valid) ok = issue_scores();
             }
             mma_commit(bar(B_DRAIN));
             bwd::drain_wait(bar(B_DRAIN), 0);
@@ -355,7 +372,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BDP_FREE));   // dP^T is in registers
             const int t0 = w.t0();
-            const uint32_t rec = stage(st) + 2 * kCTile + 32 * grp * 8;
+            const uint32_t rec = recs(st) + 32 * grp * 8;
             uint32_t pk[16], dk[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
@@ -414,25 +431,25 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(BDQ_FREE));
-                bulk_wait_group_read<0>();   // the previous reduce has read the staging tile
-            }
-            __syncwarp();
-            // staging tile = the reduce box {32 dims, 4 heads, 16 tokens}: row = chunk row,
-            // 128 bytes per row, 128-byte swizzle; lane = dim within the box
+            if (lane == 0) mbar_arrive(bar(BDQ_FREE));
+            // two reduce boxes {32 dims, 4 heads, 8 tokens} per chunk through this quarter's
+            // staging tile: row = chunk row within the box, 128 bytes per row, 128-byte
+            // swizzle; lane = dim within the box
             const uint32_t col = (uint32_t)(lane & 3) << 2;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                sts32(stg + j * 128 + ((((uint32_t)(lane >> 2)) ^ (uint32_t)(j & 7)) << 4) + col, a[j]);
+            for (int hbox = 0; hbox < 2; ++hbox) {
+                if (lane == 0) bulk_wait_group_read<0>();   // the previous reduce has read the tile
+                __syncwarp();
+                const uint32_t(&v)[32] = hbox == 0 ? a : b2;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                sts32(stg + (j + 32) * 128 + ((((uint32_t)(lane >> 2)) ^ (uint32_t)(j & 7)) << 4) + col, b2[j]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_reduce_add_4d(&tm_dq, stg, 32 * q4, wk.x.kvh * 4, wk.t0(), wk.x.b);
-                bulk_commit_group();
+                for (int j = 0; j < 32; ++j)
+                    sts32(stg + j * 128 + ((((uint32_t)(lane >> 2)) ^ (uint32_t)(j & 7)) << 4) + col, v[j]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_4d(&tm_dq, stg, 32 * q4, wk.x.kvh * 4, wk.t0() + 8 * hbox, wk.x.b);
+                    bulk_commit_group();
+                }
             }
             if (!wk.last()) continue;
             // ---- epilogue of the unit: dv, and dk through RoPE^T and the RMSNorm backward

@@ -152,6 +152,63 @@ __device__ __forceinline__ void tile_producer(const Params &p, const CUtensorMap
     for (int i = (w.g > stages ? w.g - stages : 0); i < w.g; ++i) drain_wait(full + 8 * (i % stages), (i / stages) & 1);
 }
 
+// P = 2^(S scale log2 e - mxs) of one row of a key tile (128 columns in TMEM at
+// `ts`), written as bf16 over S's first 64 columns (the P of chunk c lands on
+// S columns 16 c .. 16 c + 15, already read).  Returns the row sum.
+// kMask: columns past `hi` are masked (the unit's last key tile, which holds
+// the diagonal); the other tiles skip the compare and select, a third of the
+// per-element instructions.  kPoly: every other pair of exponentials runs on
+// the FMA pipe (exp2_poly2), which needs the exponent >= -125 -- true under
+// the fixed softmax reference, where it is >= -2 x 60.
+template <bool kPoly, bool kMask>
+__device__ __forceinline__ float softmax_tile(uint32_t ts, int hi, float sl2, float mxs)
+{
+    uint64_t sum2[2] = {0, 0};
+    const uint64_t sl2_2 = f2_pack(sl2, sl2), nm2 = f2_pack(-mxs, -mxs);
+    auto chunk = [&](const uint32_t(&v)[32], int c, uint32_t(&pk)[16]) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const uint64_t z = f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sl2_2, nm2);
+            float p0, p1;
+            if (kPoly && ((e >> 1) & 1)) {
+                const float2 r = f2_unpack(exp2_poly2(z));
+                p0 = r.x;
+                p1 = r.y;
+            } else {
+                const float2 zz = f2_unpack(z);
+                p0 = ex2(zz.x);
+                p1 = ex2(zz.y);
+            }
+            if (kMask) {
+                p0 = (32 * c + e <= hi) ? p0 : 0.f;
+                p1 = (32 * c + e + 1 <= hi) ? p1 : 0.f;
+            }
+            sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2_pack(p0, p1));
+            pk[e >> 1] = pack_bf16(p0, p1);
+        }
+    };
+    // three column chunks in flight at once, the fourth loaded into the first's
+    // registers while the second and third are computed: one TMEM load latency
+    // is exposed per tile instead of one per chunk
+    uint32_t sa[32], sb[32], sc[32], pk[16];
+    tmem_ld32(ts, sa);
+    tmem_ld32(ts + 32, sb);
+    tmem_ld32(ts + 64, sc);
+    tmem_wait_ld();
+    chunk(sa, 0, pk);
+    tmem_st16(ts, pk);
+    tmem_ld32(ts + 96, sa);
+    chunk(sb, 1, pk);
+    tmem_st16(ts + 16, pk);
+    chunk(sc, 2, pk);
+    tmem_st16(ts + 32, pk);
+    tmem_wait_ld();
+    chunk(sa, 3, pk);
+    tmem_st16(ts + 48, pk);
+    const float2 s01 = f2_unpack(f2_add(sum2[0], sum2[1]));
+    return s01.x + s01.y;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p)
@@ -231,17 +288,20 @@ full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             TileWalk w;
             w.init(p);
             bool ok = true;
+            // shared-memory descriptors built once (K-major Q~ and K~ tiles, MN-major V
+            // tiles); tiles and stages differ by constant byte offsets
+            const SmemDesc dQ = make_desc(sbase + kOffQ, 16, 1024), dK = make_desc(sbase + kOffK, 16, 1024);
+            const SmemDesc dV = make_desc(sbase + kOffV, kHalf, 1024);
             // S_X(tile g) = Q~_X K~(g)^T
             auto issue_s = [&](int x, int g, bool last) -> bool {
                 const int st = g % kKStages;
                 if (!mbar_wait(bar(BK_FULL + st), (g / kKStages) & 1, ab)) return false;
                 tc_fence_after();
-                const uint32_t qs = sbase + kOffQ + x * kTile, ks = sbase + kOffK + st * kTile;
+                const uint32_t qo = (uint32_t)x * kTile, ko = (uint32_t)st * kTile;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    mma_ss(tmem + kColS + x * 128, smem_desc_sw128(qs + off, 16, 1024),
-                           smem_desc_sw128(ks + off, 16, 1024), idesc_s, kk > 0);
+                    mma_ss(tmem + kColS + x * 128, dQ.at(qo + off), dK.at(ko + off), idesc_s, kk > 0);
                 }
                 mma_commit(bar(BS_FULL + x));
                 if (x == 1) mma_commit(bar(BK_EMPTY + st));      // tile B is the K~ stage's last reader
@@ -253,12 +313,12 @@ full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int st = g % kVStages;
                 if (!mbar_wait(bar(BV_FULL + st), (g / kVStages) & 1, ab)) return false;
                 tc_fence_after();
-                const uint32_t vs = sbase + kOffV + st * kTile;
+                const uint32_t vo = (uint32_t)st * kTile;
                 const uint32_t pa = tmem + kColS + x * 128;
+                const uint32_t acc0 = j > 0;
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk)
-                    mma_ts(tmem + kColO + x * 128, pa + kk * 8, smem_desc_sw128(vs + kk * 16 * 128, kHalf, 1024),
-                           idesc_pv, (j > 0 || kk > 0));
+                    mma_ts(tmem + kColO + x * 128, pa + kk * 8, dV.at(vo + kk * 16 * 128), idesc_pv, acc0 | (kk > 0));
                 mma_commit(bar(BPV_DONE + x));
                 if (x == 1) mma_commit(bar(BV_EMPTY + st));      // tile B is the V stage's last reader
                 return true;
@@ -378,44 +438,12 @@ full_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mxs = m_ref * p.sl2;
                 }
-                // P = 2^(S scale log2 e - reference) in bf16 over S's first 64 columns: the P
-                // of chunk c lands on S columns 16 c .. 16 c + 15, already read
-                uint64_t sum2[2] = {0, 0};
-                const uint64_t sl2_2 = f2_pack(p.sl2, p.sl2), nm2 = f2_pack(-mxs, -mxs);
-                uint32_t sa[32], sb[32];
-                tmem_ld32(ts, sa);
-#pragma unroll 1
-                for (int c = 0; c < 4; c += 2) {
-                    tmem_wait_ld();
-                    tmem_ld32(ts + 32 * (c + 1), sb);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 z = f2_unpack(f2_fma(f2_pack(__uint_as_float(sa[e]), __uint_as_float(sa[e + 1])),
-                                                          sl2_2, nm2));
-                        float p0 = ex2(z.x), p1 = ex2(z.y);
-                        p0 = (32 * c + e <= hi) ? p0 : 0.f;
-                        p1 = (32 * c + e + 1 <= hi) ? p1 : 0.f;
-                        sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2_pack(p0, p1));
-                        pk[e >> 1] = pack_bf16(p0, p1);
-                    }
-                    tmem_st16(ts + 16 * c, pk);
-                    tmem_wait_ld();
-                    if (c + 2 < 4) tmem_ld32(ts + 32 * (c + 2), sa);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 z = f2_unpack(f2_fma(f2_pack(__uint_as_float(sb[e]), __uint_as_float(sb[e + 1])),
-                                                          sl2_2, nm2));
-                        float p0 = ex2(z.x), p1 = ex2(z.y);
-                        p0 = (32 * (c + 1) + e <= hi) ? p0 : 0.f;
-                        p1 = (32 * (c + 1) + e + 1 <= hi) ? p1 : 0.f;
-                        sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], f2_pack(p0, p1));
-                        pk[e >> 1] = pack_bf16(p0, p1);
-                    }
-                    tmem_st16(ts + 16 * (c + 1), pk);
-                }
-                const float2 s01 = f2_unpack(f2_add(sum2[0], sum2[1]));
-                l += s01.x + s01.y;
+                // softmax_tile's TMEM loads and stores are warp-collective: the warp takes
+                // the masked form when any of its rows needs it
+                if (__any_sync(0xffffffffu, hi < kKeys - 1))
+                    l += softmax_tile<false, true>(ts, hi, p.sl2, mxs);   // the diagonal tile
+                else
+                    l += softmax_tile<false, false>(ts, hi, p.sl2, mxs);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();

@@ -386,7 +386,7 @@ int run_full_bwd(const gswa_shape_t *s, const void *q, const void *k, const void
         encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, kKeys) ||
         encode_bthd(&tq, qt, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
         encode_bthd(&ta, dy, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
-        encode_bthd_f32(&tdq, acc, s->B, s->T, s->Hq, s->D, 4, kChTok))
+        encode_bthd_f32(&tdq, acc, s->B, s->T, s->Hq, s->D, 4, kStgRows / 4))
         return GSWA_ERR_INVALID_ARG;
     Params p;
     std::memset(&p, 0, sizeof p);
@@ -882,7 +882,8 @@ int gswa_check_status(void *stream)
     if (v != 0) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(gswa::g_status, &zero, sizeof zero) != cudaSuccess) return GSWA_ERR_LAUNCH;
-        return v == gswa::kStatusBadArg ? GSWA_ERR_INVALID_ARG : GSWA_ERR_TIMEOUT;
+        return v == gswa::kStatusBadArg ? GSWA_ERR_INVALID_ARG
+                                        : v == gswa::kStatusSetup ? GSWA_ERR_LAUNCH : GSWA_ERR_TIMEOUT;
     }
     return GSWA_OK;
 }

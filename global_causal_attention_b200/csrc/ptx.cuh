@@ -16,6 +16,7 @@ __device__ int g_status;
 
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusBadArg = 2;   // a device-side argument (a decode position) was out of range
+constexpr int kStatusSetup = 3;    // a kernel found its launch set-up unusable (shared memory alignment)
 // A wait gives up after this much wall time (the kernels' longest legitimate
 // wait is a few microseconds; profilers that serialise passes stay far below).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
@@ -387,6 +388,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// A shared-memory descriptor kept as its two 32-bit halves, built once per
+// tile: the low half holds the start address (>> 4, 14 bits) and the leading
+// byte offset, the high half the stride byte offset and the layout bits.
+// Shared-memory addresses stay below 256 KiB, so advancing the start by a
+// constant byte offset is one 32-bit add that never carries into the leading
+// byte offset -- an MMA issue loop then spends one instruction per operand on
+// its descriptor instead of rebuilding it.
+struct SmemDesc {
+    uint32_t lo, hi;
+    __device__ __forceinline__ uint64_t at(uint32_t byte_off) const
+    {
+        uint64_t d;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo + (byte_off >> 4)), "r"(hi));
+        return d;
+    }
+};
+
+__device__ __forceinline__ SmemDesc make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    const uint64_t d = smem_desc_sw128(saddr, lbo, sbo);
+    return SmemDesc{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B, f32 accumulator.
 // a_mn/b_mn select MN-major operands (0 = K-major).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn)
@@ -477,6 +501,39 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x of a pair of floats on the FMA pipe (the softmax runs part of its
+// exponentials here so that the special-function unit, a quarter of the FMA
+// pipe's width, stops being the bound).  Cody-Waite range reduction x = j + f
+// with j = round(x) (adding 1.5 * 2^23 leaves round(x) in the low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients minimise the maximum relative error on that interval (fitted
+// by exp2_poly_fit.py: 7.5e-5, far below the bf16 rounding of P); 2^j by
+// adding j to the exponent field (the low 9 bits of 1.5 * 2^23's pattern are
+// zero, so shifting the sum's bits left by 23 leaves exactly j << 23).
+// Valid for -125 <= x <= 127.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2)
+{
+    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t t = f2_add(x2, magic);
+    const uint64_t f = f2_sub(x2, f2_sub(t, magic));
+    uint64_t p = f2_fma(f, f2_pack(0.0551712066f, 0.0551712066f), f2_pack(0.242610276f, 0.242610276f));
+    p = f2_fma(p, f, f2_pack(0.693260968f, 0.693260968f));
+    p = f2_fma(p, f, f2_pack(0.999928117f, 0.999928117f));
+    uint32_t tl, th, pl, ph;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(tl), "=r"(th) : "l"(t));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(pl), "=r"(ph) : "l"(p));
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(pl + (tl << 23)), "r"(ph + (th << 23)));
+    return r;
 }
 
 // Two floats to a packed f16 pair (`lo` in the low half), round to nearest.
