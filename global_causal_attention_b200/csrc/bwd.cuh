@@ -533,6 +533,11 @@ bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ================================================= MMA issuer
         if (lane == 0) {
             const uint32_t idesc_dq = idesc_bf16_f32(128, 128, 0, 1);
+            // shared-memory descriptors built once: Q~/dA tiles and the K~/V rings
+            // K-major, the K~ ring MN-major as the B operand of dQ~ += dS K~
+            const SmemDesc dQt = make_desc(sbase + C::kOffQ, 16, 1024), dAt = make_desc(sbase + C::kOffA, 16, 1024);
+            const SmemDesc dKr = make_desc(sbase + C::kOffK, 16, 1024), dVr = make_desc(sbase + C::kOffV, 16, 1024);
+            const SmemDesc dKmn = make_desc(sbase + C::kOffK, C::kRingHalf, 1024);
             SwaWalk ws, wd;
             ws.init(p, u0);
             wd.init(p, u0);
@@ -569,20 +574,19 @@ bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         const int n2 = kSpanBlocks - n1;
                         const uint32_t id1 = idesc_bf16_f32(128, n1 * kTok, 0, 0);
                         const uint32_t id2 = idesc_bf16_f32(128, n2 > 0 ? n2 * kTok : 32, 0, 0);
+                        const uint32_t to = (uint32_t)j * C::kTile, ro = (uint32_t)a * C::kBlockHalf;
 #pragma unroll
                         for (int op = 0; op < 2; ++op) {
                             // op 0: S from Q~ and the K~ ring; op 1: dP from dA and the V ring
                             const uint32_t dst = tmem + (op == 0 ? C::kColS : C::kColDP);
-                            const uint32_t at = sbase + (op == 0 ? C::kOffQ : C::kOffA) + j * C::kTile;
-                            const uint32_t rg = sbase + (op == 0 ? C::kOffK : C::kOffV);
+                            const SmemDesc &dt = op == 0 ? dQt : dAt;
+                            const SmemDesc &dr = op == 0 ? dKr : dVr;
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t h = kk >> 2, ko = (kk & 3) * 32;
-                                const uint64_t ad = smem_desc_sw128(at + h * C::kTileHalf + ko, 16, 1024);
-                                const uint32_t rbase = rg + h * C::kRingHalf + ko;
-                                mma_ss(dst, ad, smem_desc_sw128(rbase + a * C::kBlockHalf, 16, 1024), id1, kk > 0);
-                                if (n2 > 0)
-                                    mma_ss(dst + n1 * kTok, ad, smem_desc_sw128(rbase, 16, 1024), id2, kk > 0);
+                                const uint64_t ad = dt.at(to + h * C::kTileHalf + ko);
+                                mma_ss(dst, ad, dr.at(h * C::kRingHalf + ko + ro), id1, kk > 0);
+                                if (n2 > 0) mma_ss(dst + n1 * kTok, ad, dr.at(h * C::kRingHalf + ko), id2, kk > 0);
                             }
                         }
                         mma_commit(bar(C::BS_FULL));
@@ -606,10 +610,10 @@ bwd_dq_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const int a = dq_ring_slot(wd.s - 4);
 #pragma unroll
                     for (int kk = 0; kk < C::kSpan / 16; ++kk) {
-                        const int slot = (a + (kk >> 1)) % kRing;
-                        const uint32_t kaddr = sbase + C::kOffK + slot * C::kBlockHalf + (kk & 1) * 16 * kHalfRowBytes;
-                        mma_ts(tmem + C::kColDQ, tmem + C::kColS + kk * 8, smem_desc_sw128(kaddr, C::kRingHalf, 1024),
-                               idesc_dq, kk > 0);
+                        const int sl = a + (kk >> 1);
+                        const int slot = sl >= kRing ? sl - kRing : sl;   // a + i < 2 kRing
+                        mma_ts(tmem + C::kColDQ, tmem + C::kColS + kk * 8,
+                               dKmn.at((uint32_t)slot * C::kBlockHalf + (kk & 1) * 16 * kHalfRowBytes), idesc_dq, kk > 0);
                     }
                     mma_commit(bar(C::BS_FREE));
                     mma_commit(bar(C::BACC_FULL));
@@ -900,6 +904,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, kM, 0, 0);
             const uint32_t idesc_acc = idesc_bf16_f32(128, 128, 0, 1);
+            // shared-memory descriptors built once (stage 0; the stages differ by a
+            // constant byte offset): K~, V, P^T, dS^T and the chunk tiles K-major, the
+            // chunk tiles MN-major as the B operands of dV and dK~
+            const SmemDesc dK = make_desc(sbase + C::kOffK, 16, 1024), dV = make_desc(sbase + C::kOffV, 16, 1024);
+            const SmemDesc dP = make_desc(sbase + C::kOffP, 16, 1024), dDS = make_desc(sbase + C::kOffDS, 16, 1024);
+            const SmemDesc dC = make_desc(stage(0), 16, 1024), dCmn = make_desc(stage(0), C::kCHalf, 1024);
             KvWalk<kSwa> ws, wd;
             ws.init(p);
             wd.init(p);
@@ -912,20 +922,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
                     tc_fence_after();
                     const uint32_t dS = tmem + C::kColBuf + (ns & 1) * C::kBufStride;
-                    const uint32_t qs = stage(ns % kStages), as = qs + C::kCTile;
+                    const uint32_t qo = (uint32_t)(ns % kStages) * C::kStageBytes, ao = qo + C::kCTile;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
                         const uint32_t oc = (kk >> 2) * C::kCHalf + (kk & 3) * 32;
-                        mma_ss(dS, smem_desc_sw128(sbase + C::kOffK + ok_, 16, 1024),
-                               smem_desc_sw128(qs + oc, 16, 1024), idesc_s, kk > 0);
+                        mma_ss(dS, dK.at(ok_), dC.at(qo + oc), idesc_s, kk > 0);
                     }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
                         const uint32_t oc = (kk >> 2) * C::kCHalf + (kk & 3) * 32;
-                        mma_ss(dS + kM, smem_desc_sw128(sbase + C::kOffV + ok_, 16, 1024),
-                               smem_desc_sw128(as + oc, 16, 1024), idesc_s, kk > 0);
+                        mma_ss(dS + kM, dV.at(ok_), dC.at(ao + oc), idesc_s, kk > 0);
                     }
                     mma_commit(bar(C::BS_FULL + (ns & 1)));
                     if (ws.last()) mma_commit(bar(C::BKV_EMPTY));
@@ -936,15 +944,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (nd < ns && mbar_test(bar(C::BPS_READY), nd & 1) &&
                     (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
                     tc_fence_after();
-                    const uint32_t qs = stage(nd % kStages), as = qs + C::kCTile;
+                    const uint32_t qo = (uint32_t)(nd % kStages) * C::kStageBytes, ao = qo + C::kCTile;
+                    const uint32_t acc0 = wd.j > 0;
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
-                        mma_ss(tmem + C::kColDV, smem_desc_sw128(sbase + C::kOffP + kk * 32, 16, 1024),
-                               smem_desc_sw128(as + kk * 16 * 128, C::kCHalf, 1024), idesc_acc, (wd.j > 0 || kk > 0));
+                        mma_ss(tmem + C::kColDV, dP.at(kk * 32), dCmn.at(ao + kk * 16 * 128), idesc_acc, acc0 | (kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
-                        mma_ss(tmem + C::kColDK, smem_desc_sw128(sbase + C::kOffDS + kk * 32, 16, 1024),
-                               smem_desc_sw128(qs + kk * 16 * 128, C::kCHalf, 1024), idesc_acc, (wd.j > 0 || kk > 0));
+                        mma_ss(tmem + C::kColDK, dDS.at(kk * 32), dCmn.at(qo + kk * 16 * 128), idesc_acc, acc0 | (kk > 0));
                     mma_commit(bar(C::BCH_EMPTY + nd % kStages));
                     mma_commit(bar(C::BPS_FREE));
                     if (wd.last()) mma_commit(bar(C::BACC_FULL));

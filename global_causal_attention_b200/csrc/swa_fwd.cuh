@@ -492,6 +492,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ================================================= MMA issuer
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+            // shared-memory descriptors built once: Q tiles and the K ring K-major, the V
+            // ring MN-major (32-key blocks, halves kRingHalfBytes apart)
+            const SmemDesc dQt = make_desc(sbase + kOffQ, 16, 1024), dKr = make_desc(sbase + kOffK, 16, 1024);
+            const SmemDesc dVr = make_desc(sbase + kOffV, kRingHalfBytes, 1024);
             Walker ws, wp, wq;
             ws.init(p, u0);
             wp.init(p, u0);
@@ -535,15 +539,13 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const uint32_t id1 = idesc_bf16_f32(128, n1 * kTok, 0, 0);
                         const uint32_t id2 = idesc_bf16_f32(128, n2 > 0 ? n2 * kTok : 32, 0, 0);
                         const uint32_t dS = tmem + bb * 256;
-                        const uint32_t qs = sbase + kOffQ + bb * kTileBytes;
+                        const uint32_t qo = (uint32_t)bb * kTileBytes, ao = (uint32_t)a * kBlockHalfBytes;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t h = kk >> 2, ko = (kk & 3) * 32;
-                            const uint64_t ad = smem_desc_sw128(qs + h * kTileHalfBytes + ko, 16, 1024);
-                            const uint32_t kbase = sbase + kOffK + h * kRingHalfBytes + ko;
-                            mma_ss(dS, ad, smem_desc_sw128(kbase + a * kBlockHalfBytes, 16, 1024), id1, kk > 0);
-                            if (n2 > 0)
-                                mma_ss(dS + n1 * kTok, ad, smem_desc_sw128(kbase, 16, 1024), id2, kk > 0);
+                            const uint64_t ad = dQt.at(qo + h * kTileHalfBytes + ko);
+                            mma_ss(dS, ad, dKr.at(h * kRingHalfBytes + ko + ao), id1, kk > 0);
+                            if (n2 > 0) mma_ss(dS + n1 * kTok, ad, dKr.at(h * kRingHalfBytes + ko), id2, kk > 0);
                         }
                         mma_commit(bar(BS_FULL + bb));
                         mma_commit(bar(BQ_EMPTY + bb));
@@ -576,10 +578,11 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const uint32_t dO = tmem + bb * 256 + 128;
 #pragma unroll
                         for (int kk = 0; kk < kSpan / 16; ++kk) {
-                            const int slot = (a + (kk >> 1)) % kRing;
-                            const uint32_t vaddr = sbase + kOffV + slot * kBlockHalfBytes + (kk & 1) * 16 * kHalfRowBytes;
-                            mma_ts(dO, tmem + bb * 256 + kk * 8, smem_desc_sw128(vaddr, kRingHalfBytes, 1024),
-                                   idesc_pv, kk > 0);
+                            const int sl = a + (kk >> 1);
+                            const int slot = sl >= kRing ? sl - kRing : sl;   // a + i < 2 kRing
+                            mma_ts(dO, tmem + bb * 256 + kk * 8,
+                                   dVr.at((uint32_t)slot * kBlockHalfBytes + (kk & 1) * 16 * kHalfRowBytes), idesc_pv,
+                                   kk > 0);
                         }
                         mma_commit(bar(BO_FULL + bb));
                         // V slots that no later unit of this CTA reads
