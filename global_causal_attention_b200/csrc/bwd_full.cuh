@@ -21,23 +21,27 @@
 //   dK~ += dS^T Q~_c   (N = 128 dims)
 //   dQ~_c^T = K~^T dS^T (M = 128 dims, N = 64 rows: both operands read
 //                  transposed from the tiles already in shared memory)
-// and dQ~_c^T leaves TMEM through a swizzled shared-memory tile that a TMA
-// reduce-add sums into an f32 accumulator [B, T, Hq, D] (bwd_dq_post then
-// applies scale, RoPE^T and the RMSNorm backward).  TMEM: S buffers at 0 and
+// and dQ~_c^T leaves TMEM into registers and is added, one coalesced
+// red.global.add per chunk row and warp, into an f32 accumulator [B, T, Hq, D]
+// (bwd_dq_post then applies scale, RoPE^T and the RMSNorm backward).  TMEM: S buffers at 0 and
 // 64, dP at 128, dQ at 192, dV at 256, dK at 384 -- all 512 columns, which
 // lets the next chunk's S^T and dP^T run on the tensor pipe while the softmax
 // warps work on this one.
 //
 // dk, dv and dw_k are bitwise reproducible (fixed-order sums); the f32
-// accumulation of dq~ is not (the reduce-adds of different key tiles land in
+// accumulation of dq~ is not (the atomic adds of different key tiles land in
 // any order), and with it dq and dw_q may differ in their last bits from run
 // to run.
 //
 // Warp roles (16 warps): 0 TMA producer (K~/V once per unit; Q~, dA and the
-// row records per chunk, three stages), 1 TMEM owner and MMA issuer, 2-3 idle,
-// 4-11 softmax (two per TMEM lane quarter, 32 of the chunk's 64 rows each),
-// 12-15 dQ~ reduction and the unit epilogue (dv; dk through RoPE^T and the
-// RMSNorm backward; dw_k partials).
+// row records per chunk, four stages), 1 TMEM owner and issuer of the score
+// products (S^T, dP^T), 2 issuer of the accumulating products (dV, dK~,
+// dQ~^T), 3 idle, 4-11 softmax (two per TMEM lane quarter, 32 of the chunk's
+// 64 rows each), 12-15 dQ~ adds and the unit epilogue (dv; dk through RoPE^T
+// and the RMSNorm backward; dw_k partials).  Two issuing threads keep the
+// tensor pipe fed while either one waits on a barrier or commits: each
+// thread's commits track only the products that thread issued, and every
+// hand-off between the two goes through a barrier (below).
 #pragma once
 
 #include <cuda.h>
@@ -66,14 +70,11 @@ constexpr uint32_t kCTile = 2 * kCHalf;                   // 16 KiB
 constexpr uint32_t kStageBytes = 2 * kCTile;              // Q~ and dA of one chunk
 constexpr uint32_t kRecBytes = kChRows * 8;               // {lse log2 e, D} per row
 constexpr uint32_t kDSTile = kKeys * kHalfRowBytes;       // dS^T: 128 keys x 64 rows bf16
-constexpr int kStgRows = 32;                              // rows of one reduce box (8 tokens x 4 heads)
-constexpr uint32_t kStgBytes = kStgRows * 128;            // 32 rows x 32 dims f32
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kKTile;
 constexpr uint32_t kOffSt = kOffV + kKTile;
 constexpr uint32_t kOffDS = kOffSt + kStages * kStageBytes;
-constexpr uint32_t kOffStg = kOffDS + kDSTile;            // one staging box per TMEM lane quarter
-constexpr uint32_t kOffRec = kOffStg + 4 * kStgBytes;     // records of each stage
+constexpr uint32_t kOffRec = kOffDS + kDSTile;            // records of each stage
 constexpr uint32_t kOffW = kOffRec + kStages * kRecBytes; // f32[128] w_k
 constexpr uint32_t kOffBar = kOffW + 512;
 constexpr int kNumBars = 26;
@@ -84,24 +85,30 @@ constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 // kernel) and reports GSWA_ERR_LAUNCH through the status word otherwise.
 constexpr uint32_t kSmemBytes = kOffAbort + 4;
 static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
-static_assert((kOffSt % 1024) == 0 && (kStageBytes % 1024) == 0 && (kOffDS % 1024) == 0 && (kOffStg % 1024) == 0,
+static_assert((kOffSt % 1024) == 0 && (kStageBytes % 1024) == 0 && (kOffDS % 1024) == 0,
               "swizzled tiles are 1 KiB aligned");
 
 // TMEM columns
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 192, kColDV = 256, kColDK = 384;
 
 // Every barrier below completes at most one phase ahead of each of its
-// waiters, which is what the parity waits need.  P_READY has one barrier per S
-// buffer for that reason: the softmax warps can finish chunk g + 1 before the
-// issuer has looked at chunk g, but not chunk g + 2 (its scores are issued
-// after chunk g's accumulation).
+// waiters, which is what the parity waits need: a barrier's next phase always
+// depends, through the chain of hand-offs, on each waiter having passed its
+// wait for the current one.  P_READY and SB_FREE have one barrier per S buffer
+// for that reason: the softmax warps can finish chunk g + 1 before the
+// accumulation issuer has looked at chunk g, but not chunk g + 2 (its S^T
+// waits for chunk g's dV through SB_FREE).  Hand-offs between the two issuers:
+// SB_FREE (dV has read P^T from the S buffer the next S^T overwrites); the
+// stage and K~/V releases come from the accumulation issuer alone, whose
+// products of a chunk start only after the softmax has seen that chunk's
+// S^T and dP^T complete.
 enum : int {
     BKV_FULL = 0, BKV_EMPTY = 1, BST_FULL = 2, BST_EMPTY = BST_FULL + kStages, BS_FULL = BST_EMPTY + kStages,
     BDP_FREE = BS_FULL + 1, BP_READY = BDP_FREE + 1 /* 2 */, BSB_FREE = BP_READY + 2 /* 2 */, BDS_READY = BSB_FREE + 2,
     BDS_FREE = BDS_READY + 1, BDQ_FULL = BDS_FREE + 1, BDQ_FREE = BDQ_FULL + 1, BACC_FULL = BDQ_FREE + 1,
-    BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1
+    BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1 /* 2: one per issuer */
 };
-static_assert(B_DRAIN < kNumBars, "barrier count");
+static_assert(B_DRAIN + 1 < kNumBars, "barrier count");
 
 struct Params {
     int B, T, Tp, Hq, Hkv;
@@ -112,6 +119,7 @@ struct Params {
     const __nv_bfloat16 *k;          // raw k (RMSNorm backward)
     const __nv_bfloat16 *wk;
     __nv_bfloat16 *dk, *dv;
+    float *dq_acc;                   // [B, T, Hq, D] f32 dq~ sums (zeroed by the caller)
     float *dw_part;                  // [gridDim.x * 4][128] dw_k partials
     double theta[64];
 };
@@ -158,7 +166,7 @@ template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
-                const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ Params p)
+                const __grid_constant__ Params p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw;
@@ -195,12 +203,12 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(bar(BACC_FULL), 1);
         mbar_init(bar(BACC_FREE), 4);
         mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN + 1), 1);
         fence_barrier_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_a);
-        tma_prefetch_desc(&tm_dq);
     }
     if (tid < 128) reinterpret_cast<float *>(smem + kOffW)[tid] = __bfloat162float(p.wk[tid]);
     if (warp == 1) {
@@ -250,100 +258,87 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 bwd::drain_wait(bar(BST_FULL + i % kStages), (i / kStages) & 1);
             if (nkv > 0) bwd::drain_wait(bar(BKV_FULL), (nkv - 1) & 1);
         }
-    } else if (warp == 1) {
-        // ================================================= MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ================================================= MMA issuers
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16_f32(128, kChRows, 0, 0);     // S^T, dP^T: both K-major
             const uint32_t id_acc = idesc_bf16_f32(128, 128, 0, 1);        // dV, dK: B (rows x dims) transposed
             const uint32_t id_dq = idesc_bf16_f32(128, kChRows, 1, 1);    // dQ^T: both operands transposed
-            Walk ws, wa;   // score (S^T, dP^T) walk, one chunk ahead of the accumulate walk
-            ws.init(p);
-            wa.init(p);
-            bool ok = true;
             // shared-memory descriptors, built once: K-major (K~, V, dS^T, Q~ and dA of
             // stage 0 as A/B of the score products and dK) and MN-major (K~ as the A of
             // dQ^T; Q~, dA and dS^T as transposed B operands); the stages differ by a
             // constant byte offset
-            const SmemDesc dK_k = make_desc(sbase + kOffK, 16, 1024), dV_k = make_desc(sbase + kOffV, 16, 1024);
-            const SmemDesc dK_mn = make_desc(sbase + kOffK, kKHalf, 1024);
-            const SmemDesc dS_k = make_desc(sbase + kOffDS, 16, 1024), dS_mn = make_desc(sbase + kOffDS, kDSTile, 1024);
             const SmemDesc dC_k = make_desc(stage(0), 16, 1024), dC_mn = make_desc(stage(0), kCHalf, 1024);
-            // S^T and dP^T of chunk ws.g
-            auto issue_scores = [&]() -> bool {
-                const int g = ws.g;
-                if (ws.j == 0 && !mbar_wait(bar(BKV_FULL), ws.k & 1, ab)) return false;
-                const int st = g % kStages;
-                if (!mbar_wait(bar(BST_FULL + st), (g / kStages) & 1, ab)) return false;
-                // the S buffer's previous P^T has been read by its dV
-                if (!mbar_wait(bar(BSB_FREE + (g & 1)), ((g >> 1) & 1) ^ 1u, ab)) return false;
-                tc_fence_after();
-                const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;   // stage offsets
-                const uint32_t ds = tmem + kColS + (g & 1) * 64;
+            Walk w;
+            w.init(p);
+            bool ok = true;
+            if (warp == 1) {
+                // ---- S^T and dP^T of every chunk
+                const SmemDesc dK_k = make_desc(sbase + kOffK, 16, 1024), dV_k = make_desc(sbase + kOffV, 16, 1024);
+                for (; w.valid && ok; w.next(p)) {
+                    const int g = w.g, st = g % kStages;
+                    if (w.j == 0 && !(ok = mbar_wait(bar(BKV_FULL), w.k & 1, ab))) break;
+                    if (!(ok = mbar_wait(bar(BST_FULL + st), (g / kStages) & 1, ab))) break;
+                    // the S buffer's previous P^T (chunk g - 2) has been read by its dV
+                    if (!(ok = mbar_wait(bar(BSB_FREE + (g & 1)), ((g >> 1) & 1) ^ 1u, ab))) break;
+                    tc_fence_after();
+                    const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;   // stage offsets
+                    const uint32_t ds = tmem + kColS + (g & 1) * 64;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(ds, dK_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
-                           dC_k.at(qo + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
-                // dP: the softmax warps have loaded the previous chunk's dP^T
-                if (!mbar_wait(bar(BDP_FREE), (g & 1) ^ 1u, ab)) return false;
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(ds, dK_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
+                               dC_k.at(qo + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
+                    // dP: the softmax warps have loaded the previous chunk's dP^T
+                    if (!(ok = mbar_wait(bar(BDP_FREE), (g & 1) ^ 1u, ab))) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + kColDP, dV_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
-                           dC_k.at(ao + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
-                mma_commit(bar(BS_FULL));
-                ws.next(p);
-                return true;
-            };
-            // dV, dK and dQ^T of chunk wa.g
-            auto issue_acc = [&]() -> bool {
-                const int g = wa.g, st = g % kStages;
-                const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;
-                if (!mbar_wait(bar(BP_READY + (g & 1)), (g >> 1) & 1, ab)) return false;
-                // the first chunk of a unit overwrites dV/dK: the previous unit's epilogue has read them
-                if (wa.j == 0 && !mbar_wait(bar(BACC_FREE), (wa.k & 1) ^ 1u, ab)) return false;
-                tc_fence_after();
-                const uint32_t pt = tmem + kColS + (g & 1) * 64;
-                const uint32_t acc0 = wa.j > 0;
-#pragma unroll
-                for (int kk = 0; kk < kChRows / 16; ++kk)
-                    mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8, dC_mn.at(ao + kk * 16 * kHalfRowBytes),
-                           id_acc, acc0 | (kk > 0));
-                mma_commit(bar(BSB_FREE + (g & 1)));
-                if (!mbar_wait(bar(BDS_READY), g & 1, ab)) return false;
-                if (!mbar_wait(bar(BDQ_FREE), (g & 1) ^ 1u, ab)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kChRows / 16; ++kk)
-                    mma_ss(tmem + kColDK, dS_k.at(kk * 32), dC_mn.at(qo + kk * 16 * kHalfRowBytes), id_acc,
-                           acc0 | (kk > 0));
-#pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk)
-                    mma_ss(tmem + kColDQ, dK_mn.at(kk * 16 * kHalfRowBytes), dS_mn.at(kk * 16 * kHalfRowBytes), id_dq,
-                           kk > 0);
-                mma_commit(bar(BDQ_FULL));
-                mma_commit(bar(BDS_FREE));
-                mma_commit(bar(BST_EMPTY + st));
-                if (wa.last()) {
-                    mma_commit(bar(BACC_FULL));
-                    mma_commit(bar(BKV_EMPTY));
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + kColDP, dV_k.at((kk >> 2) * kKHalf + (kk & 3) * 32),
+                               dC_k.at(ao + (kk >> 2) * kCHalf + (kk & 3) * 32), id_s, kk > 0);
+                    mma_commit(bar(BS_FULL));
                 }
-                wa.next(p);
-                return true;
-            };
-            if (ws.valid) ok = issue_scores();
-            while (ok && wa.valid) {
-                // the next chunk's scores go ahead of this chunk's accumulation (so that
-                // its softmax overlaps these products) when its stage has landed;
-                // otherwise, and across a unit boundary (the next unit's K~/V load
-                // waits for this unit's last products), the accumulation goes first
-                const bool same_unit = ws.valid && ws.k == wa.k;
-                const bool ready = same_unit && mbar_test(bar(BST_FULL + ws.g % kStages), (ws.g / kStages) & 1);
-                if (ready) ok = issue_scores();
-                if (ok) ok = issue_acc();
-                if (ok && !ready && ws.valid) ok = issue_scores();
+            } else {
+                // ---- dV, dK~ and dQ~^T of every chunk
+                const SmemDesc dK_mn = make_desc(sbase + kOffK, kKHalf, 1024);
+                const SmemDesc dS_k = make_desc(sbase + kOffDS, 16, 1024),
+                               dS_mn = make_desc(sbase + kOffDS, kDSTile, 1024);
+                for (; w.valid && ok; w.next(p)) {
+                    const int g = w.g, st = g % kStages;
+                    const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;
+                    if (!(ok = mbar_wait(bar(BP_READY + (g & 1)), (g >> 1) & 1, ab))) break;
+                    // the first chunk of a unit overwrites dV/dK: the previous unit's epilogue has read them
+                    if (w.j == 0 && !(ok = mbar_wait(bar(BACC_FREE), (w.k & 1) ^ 1u, ab))) break;
+                    tc_fence_after();
+                    const uint32_t pt = tmem + kColS + (g & 1) * 64;
+                    const uint32_t acc0 = w.j > 0;
+#pragma unroll
+                    for (int kk = 0; kk < kChRows / 16; ++kk)
+                        mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8,
+                               dC_mn.at(ao + kk * 16 * kHalfRowBytes), id_acc, acc0 | (kk > 0));
+                    mma_commit(bar(BSB_FREE + (g & 1)));
+                    if (!(ok = mbar_wait(bar(BDS_READY), g & 1, ab))) break;
+                    if (!(ok = mbar_wait(bar(BDQ_FREE), (g & 1) ^ 1u, ab))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kChRows / 16; ++kk)
+                        mma_ss(tmem + kColDK, dS_k.at(kk * 32), dC_mn.at(qo + kk * 16 * kHalfRowBytes), id_acc,
+                               acc0 | (kk > 0));
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk)
+                        mma_ss(tmem + kColDQ, dK_mn.at(kk * 16 * kHalfRowBytes), dS_mn.at(kk * 16 * kHalfRowBytes),
+                               id_dq, kk > 0);
+                    mma_commit(bar(BDQ_FULL));
+                    mma_commit(bar(BDS_FREE));
+                    mma_commit(bar(BST_EMPTY + st));
+                    if (w.last()) {
+                        mma_commit(bar(BACC_FULL));
+                        mma_commit(bar(BKV_EMPTY));
+                    }
+                }
             }
-            mma_commit(bar(B_DRAIN));
-            bwd::drain_wait(bar(B_DRAIN), 0);
+            // this thread's products have completed before TMEM and shared memory go away
+            mma_commit(bar(B_DRAIN + (warp - 1)));
+            bwd::drain_wait(bar(B_DRAIN + (warp - 1)), 0);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
@@ -410,11 +405,11 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) mbar_arrive(bar(BDS_READY));
         }
     } else if (warp >= 12) {
-        // ================================================= dQ~ reduction, unit epilogue (4 warps)
+        // ================================================= dQ~ adds, unit epilogue (4 warps)
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;              // dQ^T: dim r; dV/dK: key r
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-        const uint32_t stg = sbase + kOffStg + q4 * kStgBytes;
+        const long long tstride = (long long)p.Hq * kD;   // accumulator floats per token
         const float *w = reinterpret_cast<const float *>(smem + kOffW);
         float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
         Walk wk;
@@ -432,24 +427,18 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BDQ_FREE));
-            // two reduce boxes {32 dims, 4 heads, 8 tokens} per chunk through this quarter's
-            // staging tile: row = chunk row within the box, 128 bytes per row, 128-byte
-            // swizzle; lane = dim within the box
-            const uint32_t col = (uint32_t)(lane & 3) << 2;
+            // dq~ += dQ~_c: chunk row c is token t0 + c / 4, head 4 kvh + c % 4; lane =
+            // dim, so each warp-wide add covers 128 contiguous bytes of one row.  Rows of
+            // tokens past T (the last chunk of a sequence) are skipped.
+            {
+                const int t0 = wk.t0();
+                const int nt = min(kChTok, p.T - t0);
+                float *dst = p.dq_acc + (((long long)wk.x.b * p.T + t0) * p.Hq + 4 * wk.x.kvh) * kD + r;
 #pragma unroll
-            for (int hbox = 0; hbox < 2; ++hbox) {
-                if (lane == 0) bulk_wait_group_read<0>();   // the previous reduce has read the tile
-                __syncwarp();
-                const uint32_t(&v)[32] = hbox == 0 ? a : b2;
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    sts32(stg + j * 128 + ((((uint32_t)(lane >> 2)) ^ (uint32_t)(j & 7)) << 4) + col, v[j]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_reduce_add_4d(&tm_dq, stg, 32 * q4, wk.x.kvh * 4, wk.t0() + 8 * hbox, wk.x.b);
-                    bulk_commit_group();
-                }
+                for (int c = 0; c < kChRows; ++c)
+                    if ((c >> 2) < nt)
+                        red_add_f32(dst + (c >> 2) * tstride + (c & 3) * kD,
+                                    __uint_as_float(c < 32 ? a[c] : b2[c - 32]));
             }
             if (!wk.last()) continue;
             // ---- epilogue of the unit: dv, and dk through RoPE^T and the RMSNorm backward
@@ -480,7 +469,6 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BACC_FREE));
         }
-        if (lane == 0) bulk_wait_group<0>();   // every reduce has completed
         float *dst = p.dw_part + ((long long)blockIdx.x * 4 + q4) * kD;
 #pragma unroll
         for (int c = 0; c < 4; ++c) dst[32 * c + lane] = dwacc[c];

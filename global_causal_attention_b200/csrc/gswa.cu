@@ -118,20 +118,6 @@ int encode_bthd(CUtensorMap *m, const void *base, int B, int T, int H, int D, in
     return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
 }
 
-// 4-D f32 tensor map over [B, T, H, D] with a {32, box_h, box_t, 1} box (one
-// 128-byte swizzled row of 32 floats per (token, head)), for reduce-adds.
-int encode_bthd_f32(CUtensorMap *m, const void *base, int B, int T, int H, int D, int box_h, int box_t)
-{
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
-    cuuint32_t box[4] = {32, (cuuint32_t)box_h, (cuuint32_t)box_t, 1};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base), dims, strides, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? GSWA_OK : GSWA_ERR_INVALID_ARG;
-}
-
 // 2-D bf16 tensor map over `rows` rows of 128 elements (a cache viewed as
 // [B * Hkv * Tmax, 128]) with a {64, box_rows} box and the 128-byte swizzle.
 int encode_rows(CUtensorMap *m, const void *base, long long rows, int box_rows)
@@ -337,11 +323,11 @@ void launch_swa_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gs
 
 template <int R>
 void launch_full_bwd(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tq, const CUtensorMap &ta,
-                     const CUtensorMap &tdq, const gswa::bwdf::Params &p, unsigned grid,
+                     const gswa::bwdf::Params &p, unsigned grid,
                      const gswa::bwdf::PostParams &pp, unsigned pgrid, cudaStream_t st)
 {
     using namespace gswa::bwdf;
-    bwd_full_kernel<R><<<grid, kThreads, kSmemBytes, st>>>(tk, tv, tq, ta, tdq, p);
+    bwd_full_kernel<R><<<grid, kThreads, kSmemBytes, st>>>(tk, tv, tq, ta, p);
     bwd_dq_post_kernel<R><<<pgrid, kPostWarps * 32, 0, st>>>(pp);
 }
 
@@ -381,12 +367,11 @@ int run_full_bwd(const gswa_shape_t *s, const void *q, const void *k, const void
 
     // 4. the fused kernel
     using namespace gswa::bwdf;
-    CUtensorMap tk, tv, tq, ta, tdq;
+    CUtensorMap tk, tv, tq, ta;
     if (encode_bthd(&tk, kt, s->B, s->T, s->Hkv, s->D, 1, kKeys) ||
         encode_bthd(&tv, v, s->B, s->T, s->Hkv, s->D, 1, kKeys) ||
         encode_bthd(&tq, qt, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
-        encode_bthd(&ta, dy, s->B, s->T, s->Hq, s->D, 4, kChTok) ||
-        encode_bthd_f32(&tdq, acc, s->B, s->T, s->Hq, s->D, 4, kStgRows / 4))
+        encode_bthd(&ta, dy, s->B, s->T, s->Hq, s->D, 4, kChTok))
         return GSWA_ERR_INVALID_ARG;
     Params p;
     std::memset(&p, 0, sizeof p);
@@ -405,6 +390,7 @@ int run_full_bwd(const gswa_shape_t *s, const void *q, const void *k, const void
     p.wk = static_cast<const __nv_bfloat16 *>(w_k);
     p.dk = static_cast<__nv_bfloat16 *>(dk);
     p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.dq_acc = static_cast<float *>(acc);
     p.dw_part = part_k;
     fill_theta(p.theta, s->rope_dims, s->rope_base);
     long long grid = p.units < num_sms ? p.units : num_sms;
@@ -429,10 +415,10 @@ int run_full_bwd(const gswa_shape_t *s, const void *q, const void *k, const void
     if (qgrid > kPostMaxGrid) qgrid = kPostMaxGrid;
 
     switch (s->rope_dims) {
-    case 0: launch_full_bwd<0>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
-    case 42: launch_full_bwd<42>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
-    case 64: launch_full_bwd<64>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
-    default: launch_full_bwd<128>(tk, tv, tq, ta, tdq, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    case 0: launch_full_bwd<0>(tk, tv, tq, ta, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    case 42: launch_full_bwd<42>(tk, tv, tq, ta, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    case 64: launch_full_bwd<64>(tk, tv, tq, ta, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
+    default: launch_full_bwd<128>(tk, tv, tq, ta, p, (unsigned)grid, q2, (unsigned)qgrid, st); break;
     }
     // 6. weight gradients, summed in a fixed order
     const unsigned rt = gswa::bwd::kD * gswa::bwd::kReduceSlices;

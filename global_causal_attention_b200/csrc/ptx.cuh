@@ -230,21 +230,12 @@ __device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src, int
         : "memory");
 }
 
-// Element-wise add of a shared-memory tile into global memory through a tensor
-// map (the tensor map's element type, here f32); the adds of different CTAs
-// to the same elements are atomic, their order unspecified.
-__device__ __forceinline__ void tma_reduce_add_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
+// Relaxed atomic add of one float to global memory, result unused (a
+// reduction at L2; a warp's 32 lanes on 32 consecutive floats make one
+// 128-byte request).
+__device__ __forceinline__ void red_add_f32(float *addr, float v)
 {
-    asm volatile(
-        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-            reinterpret_cast<uint64_t>(tmap)),
-        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
-
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a

@@ -134,7 +134,7 @@ int gswa_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void
  * (dA = dy) over every key j <= i; no g, no dg.  Layouts, workspace
  * (gswa_workspace_bytes(GSWA_OP_FULL_BWD)) and ownership as for gswa_bwd.
  * dk, dv and dw_k are bitwise reproducible; dq~ is summed in f32 by
- * reduce-adds whose order across key tiles is not fixed, so dq and dw_q may
+ * atomic adds whose order across key tiles is not fixed, so dq and dw_q may
  * differ between runs in their last bits.
  */
 int full_attn_bwd(const gswa_shape_t *shape, const void *q, const void *k, const void *v,

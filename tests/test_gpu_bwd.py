@@ -80,7 +80,7 @@ def test_full_bwd_matches_oracle(name):
 def test_bwd_deterministic():
     """The gated backward is bit-reproducible (no global atomics, fixed-order dw
     sums).  The full causal backward keeps dk, dv and dw_k bit-reproducible; its
-    dq~ is an f32 sum whose reduce-adds from different key tiles land in any
+    dq~ is an f32 sum whose atomic adds from different key tiles land in any
     order, so dq and dw_q may differ in their last bits between runs."""
     s = Shape(B=2, T=600, Hq=8, Hkv=2)
     x = {n: t.cuda() for n, t in attention_inputs(s, 20, random_weights=True, with_grad=True).items()}
