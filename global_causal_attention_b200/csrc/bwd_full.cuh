@@ -99,13 +99,19 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 192, kColDV = 256, kColDK =
 // accumulation issuer has looked at chunk g, but not chunk g + 2 (its S^T
 // waits for chunk g's dV through SB_FREE).  Hand-offs between the two issuers:
 // SB_FREE (dV has read P^T from the S buffer the next S^T overwrites); the
-// stage and K~/V releases come from the accumulation issuer alone, whose
-// products of a chunk start only after the softmax has seen that chunk's
-// S^T and dP^T complete.
+// stage and K~/V releases follow the accumulation issuer's products alone,
+// which start only after the softmax has seen that chunk's S^T and dP^T
+// complete.  The accumulation issuer waits on two barriers per chunk: P_READY,
+// and DS_READY, which counts the softmax warps' dS^T writes and the readout
+// warps' release of the previous chunk's dQ~^T columns (the readout warps
+// arrive once up front for chunk 0).  DQ_FULL, its commit after dK~ and
+// dQ~^T, tells the readout warps that dQ~^T is in TMEM, the softmax warps that dS^T
+// may be overwritten, and (through the first readout warp) the producer that
+// the chunk's stage is free.
 enum : int {
     BKV_FULL = 0, BKV_EMPTY = 1, BST_FULL = 2, BST_EMPTY = BST_FULL + kStages, BS_FULL = BST_EMPTY + kStages,
     BDP_FREE = BS_FULL + 1, BP_READY = BDP_FREE + 1 /* 2 */, BSB_FREE = BP_READY + 2 /* 2 */, BDS_READY = BSB_FREE + 2,
-    BDS_FREE = BDS_READY + 1, BDQ_FULL = BDS_FREE + 1, BDQ_FREE = BDQ_FULL + 1, BACC_FULL = BDQ_FREE + 1,
+    BDQ_FULL = BDS_READY + 1, BACC_FULL = BDQ_FULL + 1,
     BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1 /* 2: one per issuer */
 };
 static_assert(B_DRAIN + 1 < kNumBars, "barrier count");
@@ -196,10 +202,8 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(bar(BP_READY + 1), 8);
         mbar_init(bar(BSB_FREE), 1);
         mbar_init(bar(BSB_FREE + 1), 1);
-        mbar_init(bar(BDS_READY), 8);
-        mbar_init(bar(BDS_FREE), 1);
+        mbar_init(bar(BDS_READY), 8 + 4);
         mbar_init(bar(BDQ_FULL), 1);
-        mbar_init(bar(BDQ_FREE), 4);
         mbar_init(bar(BACC_FULL), 1);
         mbar_init(bar(BACC_FREE), 4);
         mbar_init(bar(B_DRAIN), 1);
@@ -303,8 +307,8 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const SmemDesc dS_k = make_desc(sbase + kOffDS, 16, 1024),
                                dS_mn = make_desc(sbase + kOffDS, kDSTile, 1024);
                 for (; w.valid && ok; w.next(p)) {
-                    const int g = w.g, st = g % kStages;
-                    const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;
+                    const int g = w.g;
+                    const uint32_t qo = (uint32_t)(g % kStages) * kStageBytes, ao = qo + kCTile;
                     if (!(ok = mbar_wait(bar(BP_READY + (g & 1)), (g >> 1) & 1, ab))) break;
                     // the first chunk of a unit overwrites dV/dK: the previous unit's epilogue has read them
                     if (w.j == 0 && !(ok = mbar_wait(bar(BACC_FREE), (w.k & 1) ^ 1u, ab))) break;
@@ -316,8 +320,8 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8,
                                dC_mn.at(ao + kk * 16 * kHalfRowBytes), id_acc, acc0 | (kk > 0));
                     mma_commit(bar(BSB_FREE + (g & 1)));
+                    // dS^T written, and the previous chunk's dQ~^T read out of TMEM
                     if (!(ok = mbar_wait(bar(BDS_READY), g & 1, ab))) break;
-                    if (!(ok = mbar_wait(bar(BDQ_FREE), (g & 1) ^ 1u, ab))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kChRows / 16; ++kk)
@@ -328,8 +332,6 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         mma_ss(tmem + kColDQ, dK_mn.at(kk * 16 * kHalfRowBytes), dS_mn.at(kk * 16 * kHalfRowBytes),
                                id_dq, kk > 0);
                     mma_commit(bar(BDQ_FULL));
-                    mma_commit(bar(BDS_FREE));
-                    mma_commit(bar(BST_EMPTY + st));
                     if (w.last()) {
                         mma_commit(bar(BACC_FULL));
                         mma_commit(bar(BKV_EMPTY));
@@ -397,7 +399,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BP_READY + (g & 1)));
             // dS^T once the previous chunk's dK and dQ^T have read the tile
-            ok = warp_wait(bar(BDS_FREE), (g & 1) ^ 1u, ab);
+            ok = warp_wait(bar(BDQ_FULL), (g & 1) ^ 1u, ab);
             if (!ok) break;
             bwd::sts_row_chunks(sbase + kOffDS, r, 4 * grp, dk);
             fence_proxy_async_smem();
@@ -415,10 +417,13 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         Walk wk;
         wk.init(p);
         bool ok = true;
+        if (lane == 0) mbar_arrive(bar(BDS_READY));   // chunk 0 has no previous dQ~^T to read out
         for (; wk.valid && ok; wk.next(p)) {
             const int g = wk.g;
             ok = warp_wait(bar(BDQ_FULL), g & 1, ab);
             if (!ok) break;
+            // the chunk's products have completed: its Q~/dA stage (and records) are free
+            if (q4 == 0 && lane == 0) mbar_arrive(bar(BST_EMPTY + g % kStages));
             tc_fence_after();
             uint32_t a[32], b2[32];
             tmem_ld32(tmem + lane_base + kColDQ, a);        // rows 0..31 of the chunk, dim r
@@ -426,7 +431,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BDQ_FREE));
+            if (lane == 0) mbar_arrive(bar(BDS_READY));   // dQ~^T columns free for the next chunk
             // dq~ += dQ~_c: chunk row c is token t0 + c / 4, head 4 kvh + c % 4; lane =
             // dim, so each warp-wide add covers 128 contiguous bytes of one row.  Rows of
             // tokens past T (the last chunk of a sequence) are skipped.
