@@ -650,7 +650,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads' device timings that the default train_4k run adds")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="run the workload at this many sequences instead of its own batch (a smaller case "
+                         "for profiler captures; the JSON line's config reports the batch used)")
     args = ap.parse_args()
+    if args.batch is not None:
+        import dataclasses
+        WORKLOADS[args.workload] = dataclasses.replace(WORKLOADS[args.workload], B=args.batch)
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]
     if args.impl == "reference":
