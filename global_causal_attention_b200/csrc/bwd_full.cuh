@@ -94,24 +94,29 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 192, kColDV = 256, kColDK =
 // Every barrier below completes at most one phase ahead of each of its
 // waiters, which is what the parity waits need: a barrier's next phase always
 // depends, through the chain of hand-offs, on each waiter having passed its
-// wait for the current one.  P_READY and SB_FREE have one barrier per S buffer
-// for that reason: the softmax warps can finish chunk g + 1 before the
-// accumulation issuer has looked at chunk g, but not chunk g + 2 (its S^T
-// waits for chunk g's dV through SB_FREE).  Hand-offs between the two issuers:
-// SB_FREE (dV has read P^T from the S buffer the next S^T overwrites); the
-// stage and K~/V releases follow the accumulation issuer's products alone,
-// which start only after the softmax has seen that chunk's S^T and dP^T
-// complete.  The accumulation issuer waits on two barriers per chunk: P_READY,
-// and DS_READY, which counts the softmax warps' dS^T writes and the readout
-// warps' release of the previous chunk's dQ~^T columns (the readout warps
-// arrive once up front for chunk 0).  DQ_FULL, its commit after dK~ and
-// dQ~^T, tells the readout warps that dQ~^T is in TMEM, the softmax warps that dS^T
-// may be overwritten, and (through the first readout warp) the producer that
-// the chunk's stage is free.
+// wait for the current one.  The accumulation issuer waits on two barriers
+// per chunk: P_READY, and DS_READY, which counts the softmax warps' dS^T
+// writes and the readout warps' release of the previous chunk's dQ~^T
+// columns (the readout warps arrive once up front for chunk 0).  It commits
+// once per chunk, DQ_FULL after dK~ and dQ~^T, which covers everything that
+// thread issued for the chunk: the readout warps learn that dQ~^T is in TMEM,
+// the softmax warps that dS^T may be overwritten, the first readout warp
+// passes the chunk's stage back to the producer, and the score issuer learns
+// that dV has read P^T out of the S buffer that chunk g + 2's scores
+// overwrite (the one hand-off between the two issuers).  P_READY and DQ_FULL
+// come in pairs, one per chunk parity (= S buffer): the score issuer waits
+// for chunk g - 2's DQ_FULL before chunk g's scores, and while it waits the
+// accumulation issuer may already finish chunk g - 1 -- on the other barrier
+// of the pair; the next phase of chunk g - 2's barrier is chunk g itself,
+// which needs those scores first.  Likewise the softmax warps can finish
+// chunk g + 1 before the accumulation issuer has looked at chunk g's
+// P_READY.  The stage and K~/V releases follow the accumulation issuer's
+// products alone, which start only after the softmax has seen that chunk's
+// S^T and dP^T complete.
 enum : int {
     BKV_FULL = 0, BKV_EMPTY = 1, BST_FULL = 2, BST_EMPTY = BST_FULL + kStages, BS_FULL = BST_EMPTY + kStages,
-    BDP_FREE = BS_FULL + 1, BP_READY = BDP_FREE + 1 /* 2 */, BSB_FREE = BP_READY + 2 /* 2 */, BDS_READY = BSB_FREE + 2,
-    BDQ_FULL = BDS_READY + 1, BACC_FULL = BDQ_FULL + 1,
+    BDP_FREE = BS_FULL + 1, BP_READY = BDP_FREE + 1 /* 2 */, BDS_READY = BP_READY + 2,
+    BDQ_FULL = BDS_READY + 1 /* 2 */, BACC_FULL = BDQ_FULL + 2,
     BACC_FREE = BACC_FULL + 1, B_DRAIN = BACC_FREE + 1 /* 2: one per issuer */
 };
 static_assert(B_DRAIN + 1 < kNumBars, "barrier count");
@@ -200,10 +205,9 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(bar(BDP_FREE), 8);
         mbar_init(bar(BP_READY), 8);
         mbar_init(bar(BP_READY + 1), 8);
-        mbar_init(bar(BSB_FREE), 1);
-        mbar_init(bar(BSB_FREE + 1), 1);
         mbar_init(bar(BDS_READY), 8 + 4);
         mbar_init(bar(BDQ_FULL), 1);
+        mbar_init(bar(BDQ_FULL + 1), 1);
         mbar_init(bar(BACC_FULL), 1);
         mbar_init(bar(BACC_FREE), 4);
         mbar_init(bar(B_DRAIN), 1);
@@ -283,8 +287,9 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int g = w.g, st = g % kStages;
                     if (w.j == 0 && !(ok = mbar_wait(bar(BKV_FULL), w.k & 1, ab))) break;
                     if (!(ok = mbar_wait(bar(BST_FULL + st), (g / kStages) & 1, ab))) break;
-                    // the S buffer's previous P^T (chunk g - 2) has been read by its dV
-                    if (!(ok = mbar_wait(bar(BSB_FREE + (g & 1)), ((g >> 1) & 1) ^ 1u, ab))) break;
+                    // the S buffer's previous P^T (chunk g - 2) has been read by its dV: chunk
+                    // g - 2's DQ_FULL commit follows that dV on the same issuing thread
+                    if (g >= 2 && !(ok = mbar_wait(bar(BDQ_FULL + (g & 1)), ((g >> 1) - 1) & 1, ab))) break;
                     tc_fence_after();
                     const uint32_t qo = (uint32_t)st * kStageBytes, ao = qo + kCTile;   // stage offsets
                     const uint32_t ds = tmem + kColS + (g & 1) * 64;
@@ -319,7 +324,6 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int kk = 0; kk < kChRows / 16; ++kk)
                         mma_ts(tmem + kColDV, pt + (kk >> 1) * 32 + (kk & 1) * 8,
                                dC_mn.at(ao + kk * 16 * kHalfRowBytes), id_acc, acc0 | (kk > 0));
-                    mma_commit(bar(BSB_FREE + (g & 1)));
                     // dS^T written, and the previous chunk's dQ~^T read out of TMEM
                     if (!(ok = mbar_wait(bar(BDS_READY), g & 1, ab))) break;
                     tc_fence_after();
@@ -331,7 +335,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int kk = 0; kk < kKeys / 16; ++kk)
                         mma_ss(tmem + kColDQ, dK_mn.at(kk * 16 * kHalfRowBytes), dS_mn.at(kk * 16 * kHalfRowBytes),
                                id_dq, kk > 0);
-                    mma_commit(bar(BDQ_FULL));
+                    mma_commit(bar(BDQ_FULL + (g & 1)));
                     if (w.last()) {
                         mma_commit(bar(BACC_FULL));
                         mma_commit(bar(BKV_EMPTY));
@@ -399,7 +403,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BP_READY + (g & 1)));
             // dS^T once the previous chunk's dK and dQ^T have read the tile
-            ok = warp_wait(bar(BDQ_FULL), (g & 1) ^ 1u, ab);
+            if (g > 0) ok = warp_wait(bar(BDQ_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1, ab);
             if (!ok) break;
             bwd::sts_row_chunks(sbase + kOffDS, r, 4 * grp, dk);
             fence_proxy_async_smem();
@@ -420,7 +424,7 @@ bwd_full_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) mbar_arrive(bar(BDS_READY));   // chunk 0 has no previous dQ~^T to read out
         for (; wk.valid && ok; wk.next(p)) {
             const int g = wk.g;
-            ok = warp_wait(bar(BDQ_FULL), g & 1, ab);
+            ok = warp_wait(bar(BDQ_FULL + (g & 1)), (g >> 1) & 1, ab);
             if (!ok) break;
             // the chunk's products have completed: its Q~/dA stage (and records) are free
             if (q4 == 0 && lane == 0) mbar_arrive(bar(BST_EMPTY + g % kStages));
