@@ -769,8 +769,8 @@ struct KvCfg {
     static constexpr int BKV_FULL = 0, BKV_EMPTY = 1, BCH_FULL = 2, BCH_EMPTY = BCH_FULL + kStages,
                          BS_FULL = BCH_EMPTY + kStages, BS_FREE = BS_FULL + 2, BPS_READY = BS_FREE + 2,
                          BPS_FREE = BPS_READY + 1, BACC_FULL = BPS_FREE + 1, BACC_FREE = BACC_FULL + 1,
-                         B_DRAIN = BACC_FREE + 1;
-    static_assert(B_DRAIN < kNumBars, "barrier count");
+                         B_DRAIN = BACC_FREE + 1 /* 2: one per issuer */;
+    static_assert(B_DRAIN + 1 < kNumBars, "barrier count");
 };
 
 struct KUnit {
@@ -846,6 +846,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(bar(C::BACC_FULL), 1);
         mbar_init(bar(C::BACC_FREE), 8);
         mbar_init(bar(C::B_DRAIN), 1);
+        mbar_init(bar(C::B_DRAIN + 1), 1);
         fence_barrier_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -899,30 +900,30 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 drain_wait(bar(C::BCH_FULL + i % kStages), (i / kStages) & 1);
             if (k > 0) drain_wait(bar(C::BKV_FULL), (k - 1) & 1);
         }
-    } else if (warp == 1) {
-        // ================================================= MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ================================================= MMA issuers: warp 1 the scores (S^T, dP^T),
+        // warp 2 the accumulations (dV, dK~); each thread's commits cover its own products
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, kM, 0, 0);
             const uint32_t idesc_acc = idesc_bf16_f32(128, 128, 0, 1);
             // shared-memory descriptors built once (stage 0; the stages differ by a
             // constant byte offset): K~, V, P^T, dS^T and the chunk tiles K-major, the
             // chunk tiles MN-major as the B operands of dV and dK~
-            const SmemDesc dK = make_desc(sbase + C::kOffK, 16, 1024), dV = make_desc(sbase + C::kOffV, 16, 1024);
-            const SmemDesc dP = make_desc(sbase + C::kOffP, 16, 1024), dDS = make_desc(sbase + C::kOffDS, 16, 1024);
             const SmemDesc dC = make_desc(stage(0), 16, 1024), dCmn = make_desc(stage(0), C::kCHalf, 1024);
-            KvWalk<kSwa> ws, wd;
-            ws.init(p);
-            wd.init(p);
-            int ns = 0, nd = 0;
-            PollWatch watch;
-            while (wd.valid) {
-                bool progressed = false;
-                if (ws.valid && ns < nd + 2 && mbar_test(bar(C::BKV_FULL), ws.k & 1) &&
-                    mbar_test(bar(C::BCH_FULL + ns % kStages), (ns / kStages) & 1) &&
-                    mbar_test(bar(C::BS_FREE + (ns & 1)), ((ns >> 1) & 1) ^ 1u)) {
+            KvWalk<kSwa> w;
+            w.init(p);
+            bool ok = true;
+            int g = 0;
+            if (warp == 1) {
+                const SmemDesc dK = make_desc(sbase + C::kOffK, 16, 1024), dV = make_desc(sbase + C::kOffV, 16, 1024);
+                for (; w.valid && ok; w.next(p), ++g) {
+                    if (w.j == 0 && !(ok = mbar_wait(bar(C::BKV_FULL), w.k & 1, ab))) break;
+                    if (!(ok = mbar_wait(bar(C::BCH_FULL + g % kStages), (g / kStages) & 1, ab))) break;
+                    // the buffer's previous scores (chunk g - 2) are in the softmax warps' registers
+                    if (!(ok = mbar_wait(bar(C::BS_FREE + (g & 1)), ((g >> 1) & 1) ^ 1u, ab))) break;
                     tc_fence_after();
-                    const uint32_t dS = tmem + C::kColBuf + (ns & 1) * C::kBufStride;
-                    const uint32_t qo = (uint32_t)(ns % kStages) * C::kStageBytes, ao = qo + C::kCTile;
+                    const uint32_t dS = tmem + C::kColBuf + (g & 1) * C::kBufStride;
+                    const uint32_t qo = (uint32_t)(g % kStages) * C::kStageBytes, ao = qo + C::kCTile;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ok_ = (kk >> 2) * C::kKHalf + (kk & 3) * 32;
@@ -935,34 +936,32 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         const uint32_t oc = (kk >> 2) * C::kCHalf + (kk & 3) * 32;
                         mma_ss(dS + kM, dV.at(ok_), dC.at(ao + oc), idesc_s, kk > 0);
                     }
-                    mma_commit(bar(C::BS_FULL + (ns & 1)));
-                    if (ws.last()) mma_commit(bar(C::BKV_EMPTY));
-                    ws.next(p);
-                    ++ns;
-                    progressed = true;
+                    mma_commit(bar(C::BS_FULL + (g & 1)));
+                    if (w.last()) mma_commit(bar(C::BKV_EMPTY));   // K~ and V are read by the scores alone
                 }
-                if (nd < ns && mbar_test(bar(C::BPS_READY), nd & 1) &&
-                    (wd.j != 0 || mbar_test(bar(C::BACC_FREE), (wd.k & 1) ^ 1u))) {
+            } else {
+                const SmemDesc dP = make_desc(sbase + C::kOffP, 16, 1024), dDS = make_desc(sbase + C::kOffDS, 16, 1024);
+                for (; w.valid && ok; w.next(p), ++g) {
+                    // P^T and dS^T of the chunk are in shared memory (the softmax warps saw
+                    // its scores complete, so the scores' reads of the stage are done)
+                    if (!(ok = mbar_wait(bar(C::BPS_READY), g & 1, ab))) break;
+                    if (w.j == 0 && !(ok = mbar_wait(bar(C::BACC_FREE), (w.k & 1) ^ 1u, ab))) break;
                     tc_fence_after();
-                    const uint32_t qo = (uint32_t)(nd % kStages) * C::kStageBytes, ao = qo + C::kCTile;
-                    const uint32_t acc0 = wd.j > 0;
+                    const uint32_t qo = (uint32_t)(g % kStages) * C::kStageBytes, ao = qo + C::kCTile;
+                    const uint32_t acc0 = w.j > 0;
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
                         mma_ss(tmem + C::kColDV, dP.at(kk * 32), dCmn.at(ao + kk * 16 * 128), idesc_acc, acc0 | (kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < kM / 16; ++kk)
                         mma_ss(tmem + C::kColDK, dDS.at(kk * 32), dCmn.at(qo + kk * 16 * 128), idesc_acc, acc0 | (kk > 0));
-                    mma_commit(bar(C::BCH_EMPTY + nd % kStages));
+                    mma_commit(bar(C::BCH_EMPTY + g % kStages));
                     mma_commit(bar(C::BPS_FREE));
-                    if (wd.last()) mma_commit(bar(C::BACC_FULL));
-                    wd.next(p);
-                    ++nd;
-                    progressed = true;
+                    if (w.last()) mma_commit(bar(C::BACC_FULL));
                 }
-                if (!watch.tick(progressed, ab)) break;
             }
-            mma_commit(bar(C::B_DRAIN));
-            drain_wait(bar(C::B_DRAIN), 0);
+            mma_commit(bar(C::B_DRAIN + (warp - 1)));
+            drain_wait(bar(C::B_DRAIN + (warp - 1)), 0);
         }
         __syncwarp();
     } else if (warp >= 4) {
