@@ -26,7 +26,7 @@ namespace dec {
 
 constexpr int kD = 128;
 constexpr int kChunk = 4096;          // keys per chunk of the full-cache split
-constexpr int kChunkWarps = 8;
+constexpr int kChunkWarps = 12;
 constexpr int kPartial = 4 + kD;      // m, l, (2 pad), o[128] per (chunk, head): o 16-byte aligned
 
 struct Params {
@@ -286,9 +286,14 @@ __device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t x, float s)
 // key reads its row without bank conflicts) by a producer warp; compute warp
 // w takes stages w, w + kChunkWarps, ... and keeps its own running (max, sum,
 // O) per head, merged at the end.  The loads of many stages are in flight at
-// once, which is what keeps HBM busy.
+// once, which is what keeps HBM busy.  There are as many stages as compute
+// warps, so warp w always reads ring slot w and waits for the phases of that
+// slot in order, each only after it has consumed the one before.  (With more
+// warps than slots a warp's first wait could target a slot's second phase
+// while its first load had not landed yet; the parity test would then take
+// the slot's earlier phase for the one wanted.)
 constexpr int kStageKeys = 32;
-constexpr int kDecStages = 12;
+constexpr int kDecStages = kChunkWarps;   // one ring slot per compute warp
 constexpr uint32_t kDecHalf = kStageKeys * 128;          // 32 keys x 64 dims bf16: 4 KiB
 constexpr uint32_t kDecTile = 2 * kDecHalf;               // one operand of a stage: 8 KiB
 constexpr uint32_t kDecStageBytes = 2 * kDecTile;          // K and V
