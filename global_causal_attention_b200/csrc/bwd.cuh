@@ -739,8 +739,11 @@ __device__ __forceinline__ void sts_row_chunks(uint32_t tile, int row, int c0, c
 // bf16 into shared memory, from where dV += P^T dA and dK~ += dS^T Q~ read
 // them.  So the next chunk's scores are computed while this chunk's
 // probabilities are formed, and every contraction runs at N >= 64 from
-// shared memory.  The same eight warps run the epilogue: dv (warps 4-7),
-// dk through RoPE^T and the RMSNorm backward (warps 8-11).
+// shared memory.  Two threads issue the MMAs (warp 1 the scores, warp 2 dV
+// and dK~), each committing only its own products.  The same eight warps run
+// the epilogue: dv (warps 4-7), dk through RoPE^T and the RMSNorm backward
+// (warps 8-11).  The sliding-window backward only: the full causal one is the
+// fused kernel of bwd_full.cuh.
 struct KvCfg {
     static constexpr int kM = 64;                    // query rows per chunk (16 tokens x 4 heads)
     static constexpr int kChTok = 16;
@@ -777,7 +780,6 @@ struct KUnit {
     int b, kvh, kt, n;   // n: query chunks of the unit
 };
 
-template <bool kSwa>
 __device__ __forceinline__ bool kv_unit_at(const Params &p, int k, KUnit &x)
 {
     const long long u = snake_unit(k);
@@ -788,30 +790,29 @@ __device__ __forceinline__ bool kv_unit_at(const Params &p, int k, KUnit &x)
     x.b = (int)(strip / p.Hkv);
     x.kvh = (int)(strip % p.Hkv);
     const int k0 = 128 * x.kt;
-    // queries that see keys [k0, k0 + 128): i in [k0, k0 + 127 + W - 1] (sliding) or [k0, T)
-    const int span = kSwa ? min(127 + p.window, p.T - k0) : p.T - k0;
+    // queries that see keys [k0, k0 + 128): i in [k0, k0 + 127 + W - 1]
+    const int span = min(127 + p.window, p.T - k0);
     x.n = (span + KvCfg::kChTok - 1) / KvCfg::kChTok;
     return true;
 }
 
-template <bool kSwa>
 struct KvWalk {
     int k = 0, j = 0;
     KUnit x;
     bool valid = false;
-    __device__ __forceinline__ void init(const Params &p) { k = 0; j = 0; valid = kv_unit_at<kSwa>(p, 0, x); }
+    __device__ __forceinline__ void init(const Params &p) { k = 0; j = 0; valid = kv_unit_at(p, 0, x); }
     __device__ __forceinline__ bool last() const { return j == x.n - 1; }
     __device__ __forceinline__ void next(const Params &p)
     {
         if (++j == x.n) {
             j = 0;
             ++k;
-            valid = kv_unit_at<kSwa>(p, k, x);
+            valid = kv_unit_at(p, k, x);
         }
     }
 };
 
-template <int R, bool kSwa>
+template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a,
@@ -870,7 +871,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             KUnit x;
             bool ok = true;
             for (; k < nunits && ok; ++k) {
-                kv_unit_at<kSwa>(p, k, x);
+                kv_unit_at(p, k, x);
                 ok = mbar_wait(bar(C::BKV_EMPTY), (k & 1) ^ 1u, ab);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(C::BKV_FULL), 2 * C::kKTile);
@@ -910,7 +911,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // constant byte offset): K~, V, P^T, dS^T and the chunk tiles K-major, the
             // chunk tiles MN-major as the B operands of dV and dK~
             const SmemDesc dC = make_desc(stage(0), 16, 1024), dCmn = make_desc(stage(0), C::kCHalf, 1024);
-            KvWalk<kSwa> w;
+            KvWalk w;
             w.init(p);
             bool ok = true;
             int g = 0;
@@ -970,13 +971,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int r = 32 * (warp & 3) + lane;      // key of the tile (TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const float *w = reinterpret_cast<const float *>(smem + C::kOffW);
-        const int W = kSwa ? p.window : (1 << 30);
+        const int W = p.window;
         float dwacc[4] = {0.f, 0.f, 0.f, 0.f};
         bool ok = true;
         int g = 0;
         KUnit x;
         for (int k = 0; k < nunits && ok; ++k) {
-            kv_unit_at<kSwa>(p, k, x);
+            kv_unit_at(p, k, x);
             const int jkey = 128 * x.kt + r;
             for (int j = 0; j < x.n && ok; ++j, ++g) {
                 const int bb = g & 1, st = g % kStages;

@@ -51,7 +51,7 @@ bool set_bwd_smem()
 {
     using namespace gswa::bwd;
     return set_smem(bwd_dq_swa_kernel<R>, DqSwaCfg::kSmemBytes) ||
-           set_smem(bwd_dkdv_kernel<R, true>, KvCfg::kSmemBytes) ||
+           set_smem(bwd_dkdv_kernel<R>, KvCfg::kSmemBytes) ||
            set_smem(gswa::bwdf::bwd_full_kernel<R>, gswa::bwdf::kSmemBytes);
 }
 
@@ -318,7 +318,7 @@ void launch_swa_bwd_main(const BwdMaps &m, const gswa::bwd::Params &pq, const gs
 {
     using namespace gswa::bwd;
     bwd_dq_swa_kernel<R><<<gq, kThreads, DqSwaCfg::kSmemBytes, st>>>(m.tq, m.ta, m.tk, m.tv, pq);
-    bwd_dkdv_kernel<R, true><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
+    bwd_dkdv_kernel<R><<<gk, kThreads, KvCfg::kSmemBytes, st>>>(m.tk2, m.tv2, m.tq2, m.ta2, pk);
 }
 
 template <int R>
