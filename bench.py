@@ -60,10 +60,10 @@ LAUNCHES = {"gswa_fwd": 2, "gswa_bwd": 7, "full_attn_fwd": 3, "full_attn_bwd": 7
 TRAFFIC = {
     ("decode_256k", "full_decode"): 34_430_000_000,  # 34.40 GB read + 0.03 GB written, 3 launches
     # one call's launches at B4 (one ncu pass), x2 for B8: each sequence's work is independent
-    ("train_4k", "gswa_fwd"): 960_400_000,
-    ("train_4k", "gswa_bwd"): 3_795_400_000,
-    ("train_4k", "full_attn_fwd"): 1_416_200_000,
-    ("train_4k", "full_attn_bwd"): 12_984_400_000,
+    ("train_4k", "gswa_fwd"): 959_200_000,
+    ("train_4k", "gswa_bwd"): 3_806_400_000,
+    ("train_4k", "full_attn_fwd"): 1_403_200_000,
+    ("train_4k", "full_attn_bwd"): 12_171_400_000,
 }
 
 
