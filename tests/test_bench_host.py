@@ -110,3 +110,26 @@ def test_stack_schedules():
     assert kinds.count("global") == 5 and kinds.count("swa") == 27
     assert kinds[30:] == ["swa", "swa"]
     assert all(st.is_global(l) == workloads.layer_is_global(l) for l in range(1, 33))
+
+
+def test_traffic_entries_name_known_workloads_and_calls():
+    """Every measured-traffic figure belongs to a workload the bench runs and
+    to one of its entry points, and is at least the call's algorithmic bytes
+    for the HBM-bound calls (ncu counts every byte moved)."""
+    for (name, op), traffic in bench.TRAFFIC.items():
+        assert name in bench.WORKLOAD_NAMES
+        assert op in bench.LAUNCHES
+        assert traffic > 0
+        if name == "train_4k":
+            bound, work, _ = bench.algorithmic_work(op, WORKLOADS["train_4k"])
+            if bound == "hbm":
+                assert traffic >= work, (op, traffic, work)
+
+
+def test_batch_override_reaches_the_reported_config(monkeypatch):
+    """--batch replaces the workload's batch, and the JSON line's config shows it."""
+    import dataclasses
+    monkeypatch.setitem(WORKLOADS, "train_4k", dataclasses.replace(WORKLOADS["train_4k"], B=4))
+    cfg = bench.workload_config("train_4k", 1)
+    assert cfg["global_batch"] == 4
+    assert "B4 T4096" in cfg["workload"]
